@@ -1,0 +1,129 @@
+"""Seeded synthetic workloads for the block-sparse attention forward.
+
+This module is shared by the CUDA path's tests and benchmark and by the
+oracle's tests.  It holds only workload *descriptions* (shapes, pattern
+parameters, seeds) and the seeded random draws of Q, K and V.  It contains
+none of the method's arithmetic: no pattern enumeration, no softmax, no
+attention.
+
+Workload recipe (stands in for the long-text corpora the pages measure on,
+which are not needed to exercise the kernel):
+
+* ``torch.Generator('cpu').manual_seed(seed)``; Q, then K, then V are drawn
+  as fp32 ``randn`` of shape [B, H, N, d] and cast to bf16 (round to nearest
+  even).
+* The local+global workload additionally draws ``u ~ U(0, 3)`` of shape
+  [B, H, N, 1] after V from the same generator and uses
+  ``K = (K_fp32 * (1 + u)).to(bf16)`` to widen the logit range.
+* ``scale = 1/sqrt(d)``.
+
+The five workloads follow the block-sparse attention pages: the log-linear
+pattern of "Block Sparse Attention with Log-Linear Complexity" (section 3.1,
+local + log-stride + 3 global anchor blocks), the Local+Global band of the
+SparseFlashAttention article (sections "Local + Global" and "Block-Sparse"),
+and the Bernoulli block mask of the RTX 4090 article ("core implementation
+logic", step 1).
+"""
+from __future__ import annotations
+
+import dataclasses
+import math
+from typing import Optional, Tuple
+
+# Pattern kinds; the numeric values are the ones of the C-ABI enum bsa_kind.
+LOGLINEAR = 0
+LOCAL_GLOBAL = 1
+BERNOULLI = 2
+
+KIND_NAMES = {LOGLINEAR: "loglinear", LOCAL_GLOBAL: "local_global", BERNOULLI: "bernoulli"}
+
+
+@dataclasses.dataclass(frozen=True)
+class PatternDesc:
+    """Plain description of a block pattern (mirrors the C struct bsa_pattern_desc)."""
+
+    kind: int
+    M: int                      # block rows = block columns = N / block_size
+    H: int                      # heads (Bernoulli differs per head; others repeat)
+    local_radius: int = 1       # LOGLINEAR: |i-j| <= radius; LOCAL_GLOBAL: band half-width w
+    log_kmax: int = 0           # LOGLINEAR: strides 2^k for k = 0..log_kmax
+    anchors: Tuple[int, ...] = ()  # LOGLINEAR: anchor columns; LOCAL_GLOBAL: full rows + columns
+    p: float = 0.0              # BERNOULLI keep probability
+    seed: int = 0               # BERNOULLI counter-based generator seed
+    causal: bool = False        # keep only columns j <= i
+
+
+@dataclasses.dataclass(frozen=True)
+class Workload:
+    name: str
+    B: int
+    H: int
+    N: int
+    d: int
+    block_size: int
+    pattern: PatternDesc
+    seed: int
+    key_scale_max: float = 0.0  # >0: K rows scaled by 1 + U(0, key_scale_max)
+    causal: bool = False        # token-level causal masking in the forward
+
+    @property
+    def M(self) -> int:
+        return self.N // self.block_size
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / math.sqrt(self.d)
+
+
+def _loglinear(M: int, H: int, kmax: int, causal: bool = False) -> PatternDesc:
+    return PatternDesc(kind=LOGLINEAR, M=M, H=H, local_radius=1, log_kmax=kmax,
+                       anchors=(0, M // 2, M - 1), causal=causal)
+
+
+WORKLOADS = {
+    # B=1 H=2 N=256 d=64 bs=32: strides k=0..2, anchors {0,4,7}
+    "tiny_loglinear": Workload("tiny_loglinear", 1, 2, 256, 64, 32, _loglinear(8, 2, 2), seed=0),
+    # B=1 H=16 N=4096 d=64 bs=32: strides k=0..6, anchors {0,64,127}
+    "loglinear_4k": Workload("loglinear_4k", 1, 16, 4096, 64, 32, _loglinear(128, 16, 6), seed=1),
+    # B=2 H=16 N=8192 d=128 bs=64: band w=4 blocks + full rows/cols 0 and M-1
+    "local_global_8k": Workload(
+        "local_global_8k", 2, 16, 8192, 128, 64,
+        PatternDesc(kind=LOCAL_GLOBAL, M=128, H=16, local_radius=4, anchors=(0, 127)),
+        seed=2, key_scale_max=3.0),
+    # B=16 H=8 N=4096 d=64 bs=64: Bernoulli(0.3) per (h, i, j), seed 7, diagonal forced
+    "bernoulli_4k": Workload(
+        "bernoulli_4k", 16, 8, 4096, 64, 64,
+        PatternDesc(kind=BERNOULLI, M=64, H=8, p=0.3, seed=7), seed=3),
+    # B=1 H=32 N=32768 d=128 bs=128: causal log-linear, strides k=0..7, anchors {0,128,255}
+    "causal_loglinear_32k": Workload(
+        "causal_loglinear_32k", 1, 32, 32768, 128, 128, _loglinear(256, 32, 7, causal=True),
+        seed=4, causal=True),
+}
+
+# The same five workloads in the order they are usually listed.
+ORDER = ["tiny_loglinear", "loglinear_4k", "local_global_8k", "bernoulli_4k", "causal_loglinear_32k"]
+
+
+def make_qkv(w: Workload, seed: Optional[int] = None):
+    """Draw bf16 Q, K, V of shape [B, H, N, d] on the CPU from the workload's seed."""
+    import torch
+
+    g = torch.Generator(device="cpu")
+    g.manual_seed(w.seed if seed is None else seed)
+    shape = (w.B, w.H, w.N, w.d)
+    q = torch.randn(shape, generator=g, dtype=torch.float32).to(torch.bfloat16)
+    k32 = torch.randn(shape, generator=g, dtype=torch.float32)
+    v = torch.randn(shape, generator=g, dtype=torch.float32).to(torch.bfloat16)
+    if w.key_scale_max > 0:
+        u = torch.rand((w.B, w.H, w.N, 1), generator=g, dtype=torch.float32) * w.key_scale_max
+        k32 = k32 * (1.0 + u)
+    k = k32.to(torch.bfloat16)
+    return q.contiguous(), k.contiguous(), v.contiguous()
+
+
+def make_qkv_shape(B: int, H: int, N: int, d: int, seed: int, key_scale_max: float = 0.0):
+    """Seeded bf16 Q, K, V for an arbitrary shape (random-shape parity sweeps)."""
+    w = Workload("adhoc", B, H, N, d, 32, PatternDesc(kind=LOGLINEAR, M=1, H=H), seed=seed,
+                 key_scale_max=key_scale_max)
+    return make_qkv(w)
+
