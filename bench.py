@@ -1,0 +1,377 @@
+"""Benchmark of the block-sparse attention forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME]
+
+One step = one bsa_forward over one batch of the workload (the whole hot
+path: one kernel launch that builds the per-tile block maps, streams Q/K/V with
+TMA, runs both contractions on tcgen05 and the restricted softmax, and writes
+O and LSE).  The pattern CSR is built once, outside the timed region.
+
+Timing: W untimed warm-up steps, then K timed steps.  The workload's inputs
+are smaller than the 126 MB L2, so before every timed step a 512 MB buffer is
+written to flush L2, and each step is bracketed by CUDA events on the
+launching stream; the reported time is the sum of the event intervals.  A
+barrier and a device synchronize surround the timed loop; with N > 1 ranks
+(torchrun) every rank runs its own replica (weak scaling, no collective in the
+data path) and the time is the max over ranks.
+
+Metric: useful TFLOP/s = 4 * bs^2 * d * (stored blocks over all heads) * B /
+time, counting every stored block in full (diagonal causal blocks included).
+
+`--impl reference` times the fp64 CPU oracle (the only reference there is) on
+the host cores, each step a bounded sample of query rows of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+METRIC = "block-sparse attn fwd useful TFLOP/s & ms/fwd (1 B200), % of roofline"
+DEFAULT_WORKLOAD = "loglinear_4k"
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+KERNEL_SOURCE = os.path.join(ROOT, "block_sparse_attention_38_b200", "csrc", "bsa_forward.cu")
+
+# DRAM bytes (read + write) per launch from ncu captures of the kernel, keyed by
+# workload, valid only for the kernel source whose sha256 prefix is given.
+NCU_TRAFFIC = {}
+
+
+def useful_flops(w, nnz_all_heads: int) -> float:
+    return 4.0 * w.block_size * w.block_size * w.d * nnz_all_heads * w.B
+
+
+def compulsory_bytes(w) -> float:
+    return 4.0 * w.B * w.H * w.N * w.d * 2 + 4.0 * w.B * w.H * w.N
+
+
+def kernel_hash() -> str:
+    with open(KERNEL_SOURCE, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def load_peaks():
+    try:
+        with open(PEAKS_FILE) as f:
+            p = json.load(f)
+        return p, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms in the background."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        import tempfile
+
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((float(parts[1]), float(parts[2]), parts[5:9]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for _, _, r in rows for i in range(4) if r[i].lower() == "active"})
+        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": reasons, "samples": len(rows)}
+
+
+def cpu_oracle_sample(w, q, k, v, rp, ci, seconds: float, rng_seed: int = 0):
+    """Time the fp64 oracle on random query rows until `seconds` of work; returns
+    (useful TFLOP/s, threads, rows done, seconds)."""
+    import oracle
+
+    rng = np.random.default_rng(rng_seed)
+    total_rows = w.B * w.H * w.N
+    lens = np.diff(rp).astype(np.int64)          # blocks per (h, block row)
+    done_rows, flops, elapsed, threads = 0, 0.0, 0.0, 0
+    batch = 256
+    while elapsed < seconds and done_rows < total_rows:
+        rows = rng.integers(0, total_rows, batch)
+        h = (rows // w.N) % w.H
+        r = (rows % w.N) // w.block_size
+        t0 = time.perf_counter()
+        _, _, threads = oracle.forward(q, k, v, rp, ci, w.block_size, w.scale, w.causal,
+                                       rows=rows)
+        elapsed += time.perf_counter() - t0
+        flops += float((4.0 * w.block_size * w.d * lens[h * w.M + r]).sum())
+        done_rows += batch
+        if elapsed < seconds / 8:
+            batch *= 2
+    return flops / elapsed / 1e12, threads, done_rows, elapsed
+
+
+def run_reference(args, w, rank, world):
+    """fp64 CPU oracle on the host cores, each step a bounded sample of rows."""
+    if rank != 0:
+        return
+    from oracle import patterns
+
+    q, k, v = workloads.make_qkv(w)
+    rp, ci = patterns.csr(w.pattern)
+    step_seconds = 2.0
+    for i in range(args.warmup):
+        cpu_oracle_sample(w, q, k, v, rp, ci, 0.2, rng_seed=1000 + i)
+    vals, times, rows_done = [], [], 0
+    threads = 0
+    for i in range(args.steps):
+        tf, threads, nrows, el = cpu_oracle_sample(w, q, k, v, rp, ci, step_seconds, rng_seed=i)
+        vals.append(tf)
+        times.append(el)
+        rows_done += nrows
+    value = statistics.median(vals)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * statistics.mean(times), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d,
+                   "block_size": w.block_size},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                         "sample": f"{rows_done} random query rows of {w.name} over {args.steps} steps"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args, w, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    import block_sparse_attention_38_b200 as bsa
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    bsa.library()
+
+    # Inputs: each rank its own replica (seed offset by rank).
+    q_h, k_h, v_h = workloads.make_qkv(w, seed=w.seed + 1000 * rank)
+    rp_np, ci_np = bsa.build_pattern_from(w.pattern)
+    nnz = int(len(ci_np))
+    flops = useful_flops(w, nnz)
+    q, k, v = q_h.to(dev), k_h.to(dev), v_h.to(dev)
+    rp = torch.from_numpy(rp_np).to(dev)
+    ci = torch.from_numpy(ci_np).to(dev)
+    O = torch.empty_like(q)
+    L = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=dev)
+    flush = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        bsa.forward(q, k, v, rp, ci, w.block_size, w.scale, w.causal, out=O, lse=L)
+
+    for _ in range(args.warmup):
+        flush.fill_(1)
+        step()
+    torch.cuda.synchronize()
+    bsa.device_status(clear=True)
+
+    visible = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+    ids = [x.strip() for x in visible.split(",") if x.strip()]
+    clocks = ClockSampler(ids[local_rank] if local_rank < len(ids) else str(local_rank))
+    if rank == 0:
+        clocks.start()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush.fill_(i & 0xFF)
+        starts[i].record(stream)
+        step()
+        ends[i].record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clock_info = clocks.stop() if rank == 0 else None
+    per_step = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    total_ms = float(sum(per_step))
+    status = bsa.device_status(clear=True)
+    if status:
+        raise RuntimeError(f"kernel reported device status {status:#x}")
+
+    # End to end through the public API: pinned host inputs -> device, forward,
+    # O and LSE back to pinned host memory, every step inside the timed region.
+    qp, kp, vp = (t.pin_memory() for t in (q_h, k_h, v_h))
+    rpp = torch.from_numpy(rp_np).pin_memory()
+    cip = torch.from_numpy(ci_np).pin_memory()
+    Oh = torch.empty(q_h.shape, dtype=torch.bfloat16).pin_memory()
+    Lh = torch.empty((w.B, w.H, w.N), dtype=torch.float32).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in (qp, kp, vp, rpp, cip))
+    d2h = Oh.numel() * Oh.element_size() + Lh.numel() * Lh.element_size()
+    qd, kd, vd = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    rpd, cid = torch.empty_like(rp), torch.empty_like(ci)
+
+    def e2e_step():
+        qd.copy_(qp, non_blocking=True)
+        kd.copy_(kp, non_blocking=True)
+        vd.copy_(vp, non_blocking=True)
+        rpd.copy_(rpp, non_blocking=True)
+        cid.copy_(cip, non_blocking=True)
+        bsa.forward(qd, kd, vd, rpd, cid, w.block_size, w.scale, w.causal, out=O, lse=L)
+        Oh.copy_(O, non_blocking=True)
+        Lh.copy_(L, non_blocking=True)
+
+    for _ in range(max(1, args.warmup)):
+        e2e_step()
+    torch.cuda.synchronize()
+    e_steps = max(3, min(args.steps, 20))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / e_steps
+
+    t_max = torch.tensor([total_ms, e2e_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t_max, op=dist.ReduceOp.MAX)
+    total_ms, e2e_ms = float(t_max[0]), float(t_max[1])
+    if rank != 0:
+        return
+
+    ms = total_ms / args.steps
+    value = flops * world / (ms * 1e-3) / 1e12
+    e2e_value = flops * world / (e2e_ms * 1e-3) / 1e12
+    peaks, peak_src = load_peaks()
+    peak_tc = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    peak_hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    t_tc = flops / (peak_tc * 1e12)
+    t_hbm = compulsory_bytes(w) / (peak_hbm * 1e9)
+    if t_tc >= t_hbm:
+        roof = {"bound": "tensor", "achieved": flops / (ms * 1e-3) / 1e12, "peak": peak_tc,
+                "unit": "TFLOP/s"}
+    else:
+        roof = {"bound": "hbm", "achieved": compulsory_bytes(w) / (ms * 1e-3) / 1e9,
+                "peak": peak_hbm, "unit": "GB/s"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    tr = NCU_TRAFFIC.get(w.name)
+    roof["traffic"] = tr[0] if tr and tr[1] == kernel_hash() else None
+    roof["peak_source"] = f"{peak_src} (MEASURED_PEAKS.json burst)" if peak_src == "measured" else "fallback"
+    roof["roofline_frac_max_of_tc_hbm"] = max(t_tc, t_hbm) / (ms * 1e-3)
+
+    # CPU baseline: the oracle, as it stands, on a bounded sample of rows.
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        from oracle import patterns
+
+        orp, oci = patterns.csr(w.pattern)
+        tf, threads, nrows, el = cpu_oracle_sample(w, q_h, k_h, v_h, orp, oci, args.cpu_seconds)
+        cpu = {"value": tf, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+               "sample": f"{nrows} random query rows of {w.name} ({el:.1f} s, fp64)"}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d,
+                   "block_size": w.block_size, "nnz_blocks": nnz, "causal": bool(w.causal),
+                   "l2": "flushed before every timed step (512 MB write)",
+                   "parallelism": f"replicas x{world}"},
+        "roofline": roof,
+        "cpu_baseline": cpu,
+        "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": int(h2d),
+                "d2h_bytes_per_step": int(d2h), "ms_per_step": e2e_ms},
+        "gpu_launches": args.steps,
+        "clocks": clock_info,
+        "min_ms": min(per_step), "median_ms": statistics.median(per_step),
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=workloads.ORDER)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    w = workloads.WORKLOADS[args.workload]
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, w, rank, world)
+        return
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        try:
+            run_ours(args, w, rank, world, local_rank)
+        finally:
+            dist.destroy_process_group()
+    else:
+        run_ours(args, w, 0, 1, 0)
+
+
+if __name__ == "__main__":
+    main()

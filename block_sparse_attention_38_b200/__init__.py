@@ -1,0 +1,179 @@
+"""B200 block-sparse attention forward: thin Python binding of libbsa.so.
+
+Every step of the computation runs in the library's C++ host code and sm_100a
+kernels; this module only marshals arguments (tensor pointers, sizes, the
+current CUDA stream) and turns non-zero status codes into exceptions.  There
+is no fallback: if libbsa.so is missing or fails to load, every call raises.
+
+    import block_sparse_attention_38_b200 as bsa
+    row_ptr, col_idx = bsa.build_pattern(bsa.LOGLINEAR, M=128, H=16, log_kmax=6,
+                                         anchors=(0, 64, 127))
+    O, LSE = bsa.forward(q, k, v, row_ptr_dev, col_idx_dev, block_size=32)
+
+The C ABI is declared in include/bsa.h.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Optional, Sequence, Tuple
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libbsa.so")
+
+# bsa_status
+OK = 0
+ERR_INVALID_ARG = -1
+ERR_UNSUPPORTED = -2
+ERR_BUFFER_TOO_SMALL = -3
+ERR_BAD_PATTERN = -4
+ERR_CUDA = -5
+STATUS_NAMES = {OK: "BSA_OK", ERR_INVALID_ARG: "BSA_ERR_INVALID_ARG",
+                ERR_UNSUPPORTED: "BSA_ERR_UNSUPPORTED",
+                ERR_BUFFER_TOO_SMALL: "BSA_ERR_BUFFER_TOO_SMALL",
+                ERR_BAD_PATTERN: "BSA_ERR_BAD_PATTERN", ERR_CUDA: "BSA_ERR_CUDA"}
+
+# bsa_kind
+LOGLINEAR = 0
+LOCAL_GLOBAL = 1
+BERNOULLI = 2
+
+# device status bits
+STATUS_TIMEOUT = 0x1
+STATUS_BAD_COLUMN = 0x2
+STATUS_BAD_ROW_PTR = 0x4
+
+
+class BsaError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        super().__init__(f"{what} failed: {STATUS_NAMES.get(code, code)}")
+        self.code = code
+
+
+class _Desc(ctypes.Structure):
+    _fields_ = [("kind", ctypes.c_int32), ("M", ctypes.c_int32), ("H", ctypes.c_int32),
+                ("local_radius", ctypes.c_int32), ("log_kmax", ctypes.c_int32),
+                ("n_anchors", ctypes.c_int32), ("anchors", ctypes.POINTER(ctypes.c_int32)),
+                ("p", ctypes.c_double), ("seed", ctypes.c_uint64), ("causal", ctypes.c_int32)]
+
+
+_lib = None
+
+
+def library() -> ctypes.CDLL:
+    """The loaded libbsa.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: build it with "
+                              "`python -m block_sparse_attention_38_b200.build`")
+        lib = ctypes.CDLL(LIB_PATH)
+        vp, i32, i64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64
+        lib.bsa_build_pattern.restype = ctypes.c_int
+        lib.bsa_build_pattern.argtypes = [ctypes.POINTER(_Desc), vp, vp, i64,
+                                          ctypes.POINTER(ctypes.c_int64)]
+        lib.bsa_validate_pattern.restype = ctypes.c_int
+        lib.bsa_validate_pattern.argtypes = [vp, vp, i64, i32, i32, i32]
+        lib.bsa_forward.restype = ctypes.c_int
+        lib.bsa_forward.argtypes = [vp, vp, vp, vp, vp, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                    ctypes.c_int, ctypes.c_int, ctypes.c_float, ctypes.c_int,
+                                    vp, vp, vp]
+        lib.bsa_device_status.restype = ctypes.c_int
+        lib.bsa_device_status.argtypes = [ctypes.POINTER(ctypes.c_uint32), ctypes.c_int]
+        lib.bsa_version.restype = ctypes.c_int
+        lib.bsa_version.argtypes = []
+        _lib = lib
+    return _lib
+
+
+def _check(code: int, what: str) -> None:
+    if code != OK:
+        raise BsaError(code, what)
+
+
+def build_pattern(kind: int, M: int, H: int, local_radius: int = 1, log_kmax: int = 0,
+                  anchors: Sequence[int] = (), p: float = 0.0, seed: int = 0,
+                  causal: bool = False) -> Tuple[np.ndarray, np.ndarray]:
+    """Block-CSR of a pattern, built on the host by bsa_build_pattern.
+
+    Returns (row_ptr int32 [H*M+1], col_idx int32 [nnz]) as numpy arrays.
+    """
+    lib = library()
+    anc = np.ascontiguousarray(np.asarray(anchors, dtype=np.int32).reshape(-1))
+    d = _Desc(int(kind), int(M), int(H), int(local_radius), int(log_kmax), int(anc.size),
+              anc.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)) if anc.size else None,
+              float(p), int(seed) & ((1 << 64) - 1), int(bool(causal)))
+    nnz = ctypes.c_int64(0)
+    _check(lib.bsa_build_pattern(ctypes.byref(d), None, None, 0, ctypes.byref(nnz)),
+           "bsa_build_pattern")
+    row_ptr = np.empty(int(H) * int(M) + 1, dtype=np.int32)
+    col_idx = np.empty(max(int(nnz.value), 1), dtype=np.int32)
+    _check(lib.bsa_build_pattern(ctypes.byref(d), row_ptr.ctypes.data, col_idx.ctypes.data,
+                                 col_idx.size, ctypes.byref(nnz)), "bsa_build_pattern")
+    return row_ptr, col_idx[: int(nnz.value)]
+
+
+def build_pattern_from(desc) -> Tuple[np.ndarray, np.ndarray]:
+    """build_pattern for any object with the bsa_pattern_desc field names."""
+    return build_pattern(desc.kind, desc.M, desc.H, desc.local_radius, desc.log_kmax,
+                         desc.anchors, desc.p, desc.seed, desc.causal)
+
+
+def validate_pattern(row_ptr: np.ndarray, col_idx: np.ndarray, H: int, M: int,
+                     causal: bool = False) -> int:
+    """Status code of bsa_validate_pattern for a host CSR (BSA_OK = 0)."""
+    rp = np.ascontiguousarray(row_ptr, dtype=np.int32)
+    ci = np.ascontiguousarray(col_idx, dtype=np.int32)
+    if rp.size != int(H) * int(M) + 1:
+        return ERR_INVALID_ARG
+    return library().bsa_validate_pattern(rp.ctypes.data, ci.ctypes.data if ci.size else None,
+                                          ci.size, int(H), int(M), int(bool(causal)))
+
+
+def forward(q, k, v, row_ptr, col_idx, block_size: int, scale: Optional[float] = None,
+            causal: bool = False, out=None, lse=None):
+    """Block-sparse attention forward through bsa_forward on q's device and current stream.
+
+    q, k, v: CUDA bf16 tensors [B, H, N, d], contiguous.  row_ptr [H*M+1] and
+    col_idx [nnz]: CUDA int32 tensors.  Returns (O bf16 [B,H,N,d], LSE fp32 [B,H,N]).
+    """
+    import torch
+
+    lib = library()
+    if q.dim() != 4 or k.shape != q.shape or v.shape != q.shape:
+        raise ValueError("q, k, v must share one shape [B, H, N, d]")
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if not t.is_cuda or t.dtype != torch.bfloat16 or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous CUDA bf16 tensor")
+    for name, t in (("row_ptr", row_ptr), ("col_idx", col_idx)):
+        if not t.is_cuda or t.dtype != torch.int32 or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous CUDA int32 tensor")
+    B, H, N, d = (int(s) for s in q.shape)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    col_ptr = col_idx.data_ptr() if col_idx.numel() else row_ptr.data_ptr()
+    with torch.cuda.device(q.device):
+        stream = torch.cuda.current_stream(q.device).cuda_stream
+        rc = lib.bsa_forward(q.data_ptr(), k.data_ptr(), v.data_ptr(), row_ptr.data_ptr(),
+                             col_ptr, B, H, N, d, int(block_size), float(scale),
+                             int(bool(causal)), out.data_ptr(), lse.data_ptr(), stream)
+    _check(rc, "bsa_forward")
+    return out, lse
+
+
+def device_status(clear: bool = True) -> int:
+    """OR of STATUS_* bits raised by kernels on the current device (synchronises it)."""
+    v = ctypes.c_uint32(0)
+    _check(library().bsa_device_status(ctypes.byref(v), int(bool(clear))), "bsa_device_status")
+    return int(v.value)
+
+
+def version() -> int:
+    return int(library().bsa_version())

@@ -1,0 +1,157 @@
+/*
+ * bsa.h -- C ABI of the B200 block-sparse attention forward.
+ *
+ * The library computes O = softmax(scale * Q K^T) V in which every query
+ * row's softmax covers only the key blocks that its block row selects
+ * ("Block Sparse Attention with Log-Linear Complexity", section 3.3: the
+ * denominator sums only over the connected K blocks; unconnected positions
+ * carry weight 0).  The block selection is a block-CSR built on the host
+ * ("precompute the index table on the CPU before the launch", section 3.2 of
+ * the same article).
+ *
+ * Conventions for every entry point:
+ *  - The caller owns all memory.  The library never allocates device memory
+ *    and never synchronises a stream.
+ *  - Argument errors are reported synchronously by the return value, with
+ *    nothing launched and nothing written.
+ *  - Q, K, V, O are bf16, [B, H, N, d] contiguous (row-major, d fastest);
+ *    LSE is fp32 [B, H, N].  Block-CSR rows are head-major: row h*M + i is
+ *    block row i of head h, M = N / block_size; the same pattern applies to
+ *    every batch entry b.
+ */
+#ifndef BSA_H
+#define BSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Status codes returned by every entry point. */
+typedef enum {
+  BSA_OK = 0,
+  BSA_ERR_INVALID_ARG = -1,      /* null pointer, non-positive size, N % block_size != 0, ... */
+  BSA_ERR_UNSUPPORTED = -2,      /* a legal value this build has no kernel for (d, block_size, M) */
+  BSA_ERR_BUFFER_TOO_SMALL = -3, /* an output buffer cannot hold the result */
+  BSA_ERR_BAD_PATTERN = -4,      /* a block-CSR violates the invariants listed at bsa_validate_pattern */
+  BSA_ERR_CUDA = -5              /* a CUDA runtime/driver call failed; cudaGetLastError() has the cause */
+} bsa_status;
+
+/* Pattern kinds. */
+typedef enum {
+  /* "Block Sparse Attention with Log-Linear Complexity", sections 2.3 and 3.1:
+   * local blocks |i-j| <= local_radius, log-stride blocks i +/- 2^k for
+   * k = 0..log_kmax (block units), and global anchor columns (anchors[]; the
+   * article names start, middle and end: 0, M/2, M-1).  Columns outside
+   * [0, M) are dropped. */
+  BSA_LOGLINEAR = 0,
+  /* SparseFlashAttention article, "Local + Global" / "Block-Sparse": band
+   * |i-j| <= local_radius, and every anchor block is a full row (it sees all
+   * blocks) and a full column (all blocks see it). */
+  BSA_LOCAL_GLOBAL = 1,
+  /* RTX 4090 article, "core implementation logic" step 1: each (h, i, j) kept
+   * with probability p, drawn from the counter-based SplitMix64 stream of
+   * `seed` (output number key+1, key = (h*M + i)*M + j, u = top 53 bits /
+   * 2^53, kept iff u < p); the diagonal is always kept. */
+  BSA_BERNOULLI = 2
+} bsa_kind;
+
+/* Pattern description (caller-owned; anchors points to n_anchors ints). */
+typedef struct {
+  int32_t kind;          /* bsa_kind */
+  int32_t M;             /* block rows = block columns, >= 1 */
+  int32_t H;             /* heads, >= 1 (LOGLINEAR / LOCAL_GLOBAL repeat one head's rows) */
+  int32_t local_radius;  /* LOGLINEAR: usually 1; LOCAL_GLOBAL: band half-width w, >= 0 */
+  int32_t log_kmax;      /* LOGLINEAR: strides 2^k for k = 0..log_kmax, 0 <= log_kmax <= 30 */
+  int32_t n_anchors;     /* number of entries in anchors, >= 0 */
+  const int32_t* anchors;/* LOGLINEAR: anchor columns; LOCAL_GLOBAL: full rows and columns;
+                            values outside [0, M) are ignored */
+  double p;              /* BERNOULLI keep probability in [0, 1] */
+  uint64_t seed;         /* BERNOULLI stream seed */
+  int32_t causal;        /* 0 or 1: keep only columns j <= i */
+} bsa_pattern_desc;
+
+/*
+ * bsa_build_pattern -- host-only, integer work only.
+ *
+ * Builds the block-CSR of `desc` over H*M rows: row_ptr[H*M+1] and the
+ * columns of every row in ascending order without repeats.
+ * Two-call use: with row_ptr == NULL and col_idx == NULL only *nnz_out is
+ * written (the number of stored blocks over all heads).  Otherwise row_ptr
+ * must hold H*M+1 ints and col_idx `cap` ints; if cap < nnz the call returns
+ * BSA_ERR_BUFFER_TOO_SMALL and writes only *nnz_out.
+ * Returns BSA_ERR_INVALID_ARG for a null desc/nnz_out, M < 1, H < 1, an
+ * unknown kind, a negative radius, log_kmax outside [0, 30], p outside
+ * [0, 1], n_anchors < 0 or anchors == NULL with n_anchors > 0, causal not
+ * 0/1, or an nnz that does not fit int32.
+ */
+int bsa_build_pattern(const bsa_pattern_desc* desc, int32_t* row_ptr, int32_t* col_idx,
+                      int64_t cap, int64_t* nnz_out);
+
+/*
+ * bsa_validate_pattern -- host-only check of a block-CSR held in host memory.
+ *
+ * Checks: row_ptr[0] == 0; row_ptr non-decreasing; row_ptr[H*M] <= col_cap
+ * (else BSA_ERR_BUFFER_TOO_SMALL); every column in [0, M); columns strictly
+ * ascending within a row; with causal == 1 every column j of block row i has
+ * j <= i.  Returns BSA_OK or BSA_ERR_BAD_PATTERN (BSA_ERR_INVALID_ARG for
+ * null pointers or non-positive H, M).
+ */
+int bsa_validate_pattern(const int32_t* row_ptr, const int32_t* col_idx, int64_t col_cap,
+                         int32_t H, int32_t M, int32_t causal);
+
+/*
+ * bsa_forward -- the block-sparse attention forward on the current CUDA
+ * device, enqueued on `stream` (a cudaStream_t; NULL = legacy default).
+ *
+ * For batch b, head h and query token q of block row r = q / block_size:
+ *   keys(q) = tokens of the blocks col_idx[row_ptr[h*M+r] .. row_ptr[h*M+r+1])
+ *             minus the tokens k > q when causal == 1;
+ *   O[b,h,q,:] = sum_k softmax_k(scale * Q[b,h,q,:] . K[b,h,k,:]) V[b,h,k,:]
+ *   LSE[b,h,q] = ln sum_k exp(scale * Q[b,h,q,:] . K[b,h,k,:])   (natural log)
+ *   An empty keys(q) gives O = 0 and LSE = -inf.
+ * Inputs bf16, products and sums in fp32 on the tensor cores, softmax
+ * statistics in fp32, O rounded to bf16 (nearest even).
+ *
+ * Q, K, V, O: device pointers, bf16 [B,H,N,d] contiguous, 16-byte aligned.
+ * LSE: device pointer, fp32 [B,H,N], 16-byte aligned.  O and LSE must not
+ * overlap the inputs.
+ * row_ptr: device int32 [H*M+1]; col_idx: device int32 [row_ptr[H*M]].
+ * The columns of a row may come in any order; a repeated column counts once.
+ * Columns outside [0, M) are skipped and flagged in the device status word
+ * (bsa_device_status).  row_ptr must be non-decreasing and col_idx must hold
+ * row_ptr[H*M] entries: the call does not read the CSR on the host (use
+ * bsa_validate_pattern there).
+ * Supported: d in {64, 128}; block_size in {32, 64, 128}; N % block_size == 0;
+ * 1 <= M <= 4096; B*H <= 2^31-1.  Else BSA_ERR_INVALID_ARG /
+ * BSA_ERR_UNSUPPORTED, nothing launched.  A failed launch returns BSA_ERR_CUDA.
+ * The call returns without synchronising.
+ */
+int bsa_forward(const void* Q, const void* K, const void* V,
+                const int32_t* row_ptr, const int32_t* col_idx,
+                int B, int H, int N, int d, int block_size, float scale, int causal,
+                void* O, float* LSE, void* stream);
+
+/* Bits of the device status word. */
+#define BSA_STATUS_TIMEOUT     0x1u  /* a bounded wait inside the kernel gave up */
+#define BSA_STATUS_BAD_COLUMN  0x2u  /* a column index outside [0, M) was skipped */
+#define BSA_STATUS_BAD_ROW_PTR 0x4u  /* row_ptr[i+1] < row_ptr[i] was seen; the row was treated as empty */
+
+/*
+ * bsa_device_status -- read (and with clear != 0, reset) the status word of
+ * the current device.  Synchronises the device.  Returns BSA_OK or
+ * BSA_ERR_CUDA; *status receives an OR of BSA_STATUS_* bits accumulated by
+ * the kernels since the last clear.
+ */
+int bsa_device_status(uint32_t* status, int clear);
+
+/* Library version as an integer (major*10000 + minor*100 + patch). */
+int bsa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BSA_H */
