@@ -138,7 +138,7 @@ def cpu_oracle_sample(w, q, k, v, rp, ci, seconds: float, rng_seed: int = 0):
     lens = np.diff(rp).astype(np.int64)          # blocks per (h, block row)
     done_rows, flops, elapsed, threads = 0, 0.0, 0.0, 0
     batch = 256
-    while elapsed < seconds and done_rows < total_rows:
+    while elapsed < seconds:
         rows = rng.integers(0, total_rows, batch)
         h = (rows // w.N) % w.H
         r = (rows % w.N) // w.block_size
