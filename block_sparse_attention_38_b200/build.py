@@ -18,7 +18,8 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 SOURCES = [os.path.join(CSRC, "bsa_pattern.cpp"), os.path.join(CSRC, "bsa_forward.cu")]
-DEPS = SOURCES + [os.path.join(CSRC, "sm100_ptx.cuh"), os.path.join(ROOT, "include", "bsa.h")]
+DEPS = SOURCES + [os.path.join(CSRC, f) for f in sorted(os.listdir(CSRC)) if f.endswith(".cuh")] + [
+    os.path.join(ROOT, "include", "bsa.h")]
 LIB = os.path.join(HERE, "libbsa.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 

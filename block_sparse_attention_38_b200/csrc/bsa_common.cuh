@@ -1,0 +1,104 @@
+// bsa_common.cuh -- definitions shared by the forward kernels: the device
+// status word, the launch arguments, bounded mbarrier waits and a bitmap
+// iterator.  Included once, by bsa_forward.cu (a single translation unit).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+
+#include "../../include/bsa.h"
+#include "sm100_ptx.cuh"
+
+namespace bsa {
+
+
+constexpr int kMaxM = 4096;                 // block rows supported per head
+constexpr int kMaxBitmapWords = kMaxM / 32;
+constexpr float kRescaleThreshold = 8.0f;   // log2 units: O is rescaled only when the max grows by > 2^8
+constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s: a wait longer than this is a hang
+
+__device__ unsigned int g_status;
+
+struct FwdArgs {
+  const int32_t* row_ptr;
+  const int32_t* col_idx;
+  __nv_bfloat16* O;
+  float* LSE;
+  int H, N, M, G, W;      // G = tiles per (b, h); W = 32-bit words per block-row bitmap
+  long long num_tiles;
+  float scale_log2;       // scale * log2(e)
+  int causal;
+};
+
+struct AbortFlag {
+  volatile int v;
+};
+
+// Bounded wait: true when the phase of parity `parity` has completed; false
+// after kWaitLimitNs or when another warp has already given up.
+__device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, AbortFlag* ab) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 63u) == 0) {
+      if (ab->v) return false;
+      if (global_timer_ns() - t0 > kWaitLimitNs) {
+        ab->v = 1;
+        atomicOr(&g_status, BSA_STATUS_TIMEOUT);
+        return false;
+      }
+    }
+  }
+}
+
+// Same, for teardown: ignores the abort flag (used to drain copies already in flight).
+__device__ __forceinline__ void wait_drain(uint64_t* bar, uint32_t parity) {
+  const uint64_t t0 = global_timer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (global_timer_ns() - t0 > kWaitLimitNs) {
+      atomicOr(&g_status, BSA_STATUS_TIMEOUT);
+      return;
+    }
+  }
+}
+
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, AbortFlag* ab) {
+  const bool ok = wait_bounded(bar, parity, ab);
+  return __all_sync(0xffffffffu, ok);
+}
+
+__device__ __forceinline__ int union_count(const uint32_t* uni, int W) {
+  int n = 0;
+  for (int w = 0; w < W; ++w) n += __popc(uni[w]);
+  return n;
+}
+
+// Walks the set bits of a bitmap in ascending order.
+struct BitIter {
+  const uint32_t* bits;
+  int W, w;
+  uint32_t cur;
+  __device__ __forceinline__ BitIter(const uint32_t* b, int W_) : bits(b), W(W_), w(0), cur(b[0]) {}
+  __device__ __forceinline__ int next() {
+    while (cur == 0) {
+      if (++w >= W) return -1;
+      cur = bits[w];
+    }
+    const int b = __ffs(cur) - 1;
+    cur &= cur - 1;
+    return w * 32 + b;
+  }
+};
+
+
+// Named barrier over `nthreads` threads (ids 1..15; id 0 is __syncthreads).
+__device__ __forceinline__ void named_bar(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+}  // namespace bsa

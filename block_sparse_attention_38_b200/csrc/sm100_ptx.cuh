@@ -144,20 +144,32 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn_ma
          (static_cast<uint32_t>(M >> 4) << 24);
 }
 
-// Shared-memory matrix descriptor for the 128-byte swizzle (PTX ISA, "Shared
-// memory descriptor"): bits 0-13 start address >> 4, 16-29 leading-dimension
-// byte offset >> 4, 32-45 stride-dimension byte offset >> 4, 46-47 version
-// (1 on sm_100), 61-63 layout (2 = 128-byte swizzle).  The swizzle atom is
-// 8 rows x 128 bytes and must start on a 1024-byte boundary.
-__device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo_bytes,
-                                                uint32_t sbo_bytes) {
+// Shared-memory matrix descriptor (PTX ISA, "Shared memory descriptor"):
+// bits 0-13 start address >> 4, 16-29 leading-dimension byte offset >> 4,
+// 32-45 stride-dimension byte offset >> 4, 46-47 version (1 on sm_100),
+// 61-63 layout (kLayoutSW128 = 2: 128-byte swizzle, atom 8 rows x 128 B on a
+// 1024-byte boundary; kLayoutSW64 = 4: 64-byte swizzle, atom 8 rows x 64 B on
+// a 512-byte boundary).
+// K-major swizzled operands: SBO = byte distance between 8-row groups; LBO unused.
+// MN-major swizzled operands: LBO = byte distance between swizzle-atom columns
+// along M/N, SBO = byte distance between 8-row groups along K.
+constexpr uint32_t kLayoutSW128 = 2;
+constexpr uint32_t kLayoutSW64 = 4;
+
+__device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes,
+                                          uint32_t layout) {
   uint64_t d = 0;
   d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
   d |= static_cast<uint64_t>((lbo_bytes >> 4) & 0x3FFFu) << 16;
   d |= static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFFu) << 32;
   d |= static_cast<uint64_t>(1) << 46;
-  d |= static_cast<uint64_t>(2) << 61;
+  d |= static_cast<uint64_t>(layout & 7u) << 61;
   return d;
+}
+
+__device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo_bytes,
+                                                uint32_t sbo_bytes) {
+  return sdesc(saddr, lbo_bytes, sbo_bytes, kLayoutSW128);
 }
 
 // ------------------------------------------------------------------- math

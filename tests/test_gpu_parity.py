@@ -145,6 +145,32 @@ def test_random_patterns(shape, causal):
     _compare(O, L, Or, Lr, str(shape))
 
 
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("bs", [32, 64, 128])
+def test_many_tiles_per_cta_varying_row_lengths(bs, d):
+    # more tiles than SMs, so every CTA walks several tiles and reuses its
+    # rings and buffers; band edges and random rows give many partial chunks
+    B, H, N = 1, 16, 4096 if bs == 32 else 8192
+    M = N // bs
+    rng = np.random.default_rng(bs * 1000 + d)
+    rows = []
+    for h in range(H):
+        for i in range(M):
+            w = int(rng.integers(0, 4))
+            cols = [j for j in range(i - w, i + w + 1) if 0 <= j < M]
+            cols += [int(x) for x in rng.integers(0, M, int(rng.integers(0, 6)))]
+            rows.append(sorted(set(cols)))
+    rp = np.zeros(H * M + 1, np.int32)
+    rp[1:] = np.cumsum([len(r) for r in rows])
+    ci = np.array([j for r in rows for j in r], np.int32)
+    q, k, v = workloads.make_qkv_shape(B, H, N, d, seed=bs + d)
+    O, L = _run_gpu(q, k, v, rp, ci, bs, 1.0 / math.sqrt(d), False)
+    assert bsa.device_status(clear=True) == 0
+    rows_s = np.unique(np.concatenate([np.arange(0, 2 * N), rng.integers(0, B * H * N, 4096)]))
+    Or, Lr, _ = oracle.forward(q, k, v, rp, ci, bs, 1.0 / math.sqrt(d), False, rows=rows_s)
+    _compare(O.reshape(-1, d)[rows_s], L.reshape(-1)[rows_s], Or, Lr, f"bs={bs} d={d}")
+
+
 def test_all_rows_empty():
     B, H, N, d, bs = 1, 2, 256, 64, 32
     q, k, v = workloads.make_qkv_shape(B, H, N, d, seed=5)
@@ -153,18 +179,22 @@ def test_all_rows_empty():
     assert np.all(O == 0.0) and np.all(np.isneginf(L))
 
 
-def test_dense_pattern_large_logits_and_causal():
-    # every block present, K scaled up: the running max moves often and far
-    B, H, N, d, bs = 1, 2, 512, 128, 64
+@pytest.mark.parametrize("bs,d,N", [(32, 64, 1024), (32, 128, 2048), (64, 128, 512), (128, 64, 1024)])
+def test_dense_pattern_large_logits_and_causal(bs, d, N):
+    # every block present, K scaled up: the running max moves often and far.
+    # At block_size 32 a row of 32+ blocks spans several TMEM-resident groups
+    # of chunks, so the rescaling between groups is exercised too.
+    B, H = 1, 2
     M = N // bs
-    q, k, v = workloads.make_qkv_shape(B, H, N, d, seed=8)
+    q, k, v = workloads.make_qkv_shape(B, H, N, d, seed=8 + bs)
     k = (k.float() * 6).to(torch.bfloat16)
     rp = np.arange(0, H * M * M + 1, M, dtype=np.int32)
     ci = np.tile(np.arange(M, dtype=np.int32), H * M)
     for causal in (False, True):
         O, L = _run_gpu(q, k, v, rp, ci, bs, 1.0 / math.sqrt(d), causal)
+        assert bsa.device_status(clear=True) == 0
         Or, Lr, _ = oracle.forward(q, k, v, rp, ci, bs, 1.0 / math.sqrt(d), causal)
-        _compare(O, L, Or, Lr, f"dense causal={causal}")
+        _compare(O, L, Or, Lr, f"dense bs={bs} causal={causal}")
         ref = torch.nn.functional.scaled_dot_product_attention(
             q.float(), k.float(), v.float(), is_causal=causal, scale=1.0 / math.sqrt(d))
         assert float((torch.from_numpy(O) - ref).abs().max()) <= O_MAX
