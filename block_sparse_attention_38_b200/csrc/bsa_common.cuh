@@ -10,7 +10,7 @@
 #include <cmath>
 #include <cstdint>
 
-#include "../../include/bsa.h"
+#include "bsa.h"
 #include "sm100_ptx.cuh"
 
 namespace bsa {
@@ -19,13 +19,16 @@ namespace bsa {
 constexpr int kMaxM = 4096;                 // block rows supported per head
 constexpr int kMaxBitmapWords = kMaxM / 32;
 constexpr float kRescaleThreshold = 8.0f;   // log2 units: O is rescaled only when the max grows by > 2^8
-constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s: a wait longer than this is a hang
+constexpr long long kWaitLimitCycles = 4000000000LL;  // ~2 s at 1.97 GHz: a longer wait is a hang
 
 __device__ unsigned int g_status;
 
 struct FwdArgs {
   const int32_t* row_ptr;
   const int32_t* col_idx;
+  const __nv_bfloat16* Q;  // [B,H,N,d] (read with cp.async by the key-tile kernel)
+  const __nv_bfloat16* K;
+  const __nv_bfloat16* V;
   __nv_bfloat16* O;
   float* LSE;
   int H, N, M, G, W;      // G = tiles per (b, h); W = 32-bit words per block-row bitmap
@@ -39,15 +42,21 @@ struct AbortFlag {
 };
 
 // Bounded wait: true when the phase of parity `parity` has completed; false
-// after kWaitLimitNs or when another warp has already given up.
+// once about kWaitLimitCycles SM cycles have passed (>= 2 s at the B200's top
+// clock) or when another warp has already given up.  The cycle counter is read
+// only every 1024 polls so that a phase completing during the wait is seen
+// within one try_wait.
 __device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, AbortFlag* ab) {
   if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = global_timer_ns();
+  long long t0 = 0;
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 63u) == 0) {
+    if ((it & 1023u) == 0) {
       if (ab->v) return false;
-      if (global_timer_ns() - t0 > kWaitLimitNs) {
+      const long long now = clock64();
+      if (t0 == 0) {
+        t0 = now;
+      } else if (now - t0 > kWaitLimitCycles) {
         ab->v = 1;
         atomicOr(&g_status, BSA_STATUS_TIMEOUT);
         return false;
@@ -58,9 +67,9 @@ __device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, Abo
 
 // Same, for teardown: ignores the abort flag (used to drain copies already in flight).
 __device__ __forceinline__ void wait_drain(uint64_t* bar, uint32_t parity) {
-  const uint64_t t0 = global_timer_ns();
-  while (!mbar_try_wait(bar, parity)) {
-    if (global_timer_ns() - t0 > kWaitLimitNs) {
+  const long long t0 = clock64();
+  for (uint32_t it = 0; !mbar_try_wait(bar, parity); ++it) {
+    if ((it & 1023u) == 1023u && clock64() - t0 > kWaitLimitCycles) {
       atomicOr(&g_status, BSA_STATUS_TIMEOUT);
       return;
     }
@@ -97,8 +106,11 @@ struct BitIter {
 
 
 // Named barrier over `nthreads` threads (ids 1..15; id 0 is __syncthreads).
+// The warp is reconverged first and the non-aligned form is used, so a lane
+// that arrives after a divergent branch of its warp still counts correctly.
 __device__ __forceinline__ void named_bar(int id, int nthreads) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+  __syncwarp();
+  asm volatile("barrier.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
 }  // namespace bsa

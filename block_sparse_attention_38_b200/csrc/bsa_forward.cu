@@ -85,6 +85,8 @@ int launch_rows(const void* Q, const void* K, const void* V, const int32_t* row_
   FwdArgs a;
   a.row_ptr = row_ptr;
   a.col_idx = col_idx;
+  a.K = static_cast<const __nv_bfloat16*>(K);
+  a.V = static_cast<const __nv_bfloat16*>(V);
   a.O = static_cast<__nv_bfloat16*>(O);
   a.LSE = LSE;
   a.H = H;
@@ -121,13 +123,12 @@ int launch_keys(const void* Q, const void* K, const void* V, const int32_t* row_
   DeviceInfo di;
   if (!device_info(dev, &di)) return BSA_ERR_CUDA;
   const long long BH = static_cast<long long>(B) * H;
-  CUtensorMap tq, tk, tv;
-  if (!make_map(&tq, Q, BH, N, D, 32) || !make_map(&tk, K, BH, N, D, 32) ||
-      !make_map(&tv, V, BH, N, D, 32))
-    return BSA_ERR_CUDA;
   FwdArgs a;
   a.row_ptr = row_ptr;
   a.col_idx = col_idx;
+  a.Q = static_cast<const __nv_bfloat16*>(Q);
+  a.K = static_cast<const __nv_bfloat16*>(K);
+  a.V = static_cast<const __nv_bfloat16*>(V);
   a.O = static_cast<__nv_bfloat16*>(O);
   a.LSE = LSE;
   a.H = H;
@@ -146,8 +147,9 @@ int launch_keys(const void* Q, const void* K, const void* V, const int32_t* row_
       return BSA_ERR_CUDA;
     attr_set[dev] = true;
   }
-  const long long grid = a.num_tiles < di.sms ? a.num_tiles : di.sms;
-  keys::fwd_kernel<D><<<static_cast<unsigned>(grid), keys::kThreads, smem, stream>>>(tq, tk, tv, a);
+  const long long pipes = (a.num_tiles + C::NWG - 1) / C::NWG;
+  const long long grid = pipes < di.sms ? pipes : di.sms;
+  keys::fwd_kernel<D><<<static_cast<unsigned>(grid), C::THREADS, smem, stream>>>(a);
   if (cudaGetLastError() != cudaSuccess) return BSA_ERR_CUDA;
   return BSA_OK;
 }

@@ -6,31 +6,39 @@
 // coincide), so a tile of four block rows would compute their union, about
 // 2.5 times the useful work.  This kernel puts the *keys* on M instead:
 //
-//   tile  = one block row (b, h, r): 32 queries, its L column blocks;
-//   chunk = 4 of those column blocks gathered by TMA into 128 key rows;
+//   tile  = one block row (b, h, r): 32 queries and its L column blocks;
+//   chunk = 4 of those column blocks gathered into 128 key rows;
 //   S^T   = K_chunk Q^T          (M=128 keys, N=32 queries, K=d) -> TMEM;
 //   O^T  += V_chunk^T P^T        (M=d rows, N=32 queries, K=128 keys) -> TMEM.
 //
 // Thread t of a softmax warpgroup owns key row t of a chunk and reads its 32
-// query scores with one tcgen05.ld.  The restricted softmax ("Block Sparse
-// Attention with Log-Linear Complexity", section 3.3: the denominator sums
-// only over the connected key blocks) needs per-query statistics across key
-// rows, so they come from a warp transpose-reduction (31 shuffles for 32
-// queries) plus a 4-warp exchange in shared memory, once per group of up to
-// kChunksResident chunks kept in TMEM: pass 1 takes the exact row maximum,
-// pass 2 writes P^T = 2^(s - max) in bf16 and accumulates the fp32 row sums,
-// which are transpose-reduced once per tile.  For d = 64 the O^T MMA still
-// uses M = 128 (the single-CTA shape whose TMEM layout is one row per lane):
-// the upper 64 rows of its A operand are a constant zero tile and rows
-// 64..127 of O^T are ignored.  Rows longer than kChunksResident chunks are
-// processed in groups with the usual rescaling of O^T and the sums between
-// groups.
+// query scores with one tcgen05.ld.  The softmax is restricted to the
+// connected key blocks ("Block Sparse Attention with Log-Linear Complexity",
+// section 3.3: the denominator sums only over them).  It runs in one pass per
+// chunk with a lazily updated maximum: p = 2^(s - m) with the current
+// per-query maximum m as long as no score exceeds m by more than 2^8 (a
+// warpgroup-wide vote per chunk); otherwise -- always on a row's first chunk
+// -- the exact per-query maximum is formed by a warp transpose-reduction (31
+// shuffles for 32 queries) and a 4-warp exchange in shared memory, and O^T
+// and the row sums are rescaled.  Row sums are kept in fp32 per thread and
+// reduced once per tile.  For d = 64 the O^T MMA still uses M = 128 (the
+// single-CTA shape whose TMEM layout is one row per lane): the upper 64 rows
+// of its A operand are a constant zero tile and rows 64..127 of O^T are
+// ignored.
 //
-// Warps: 0-3 and 4-7 are two softmax warpgroups working on alternate tiles
-// (each with its own TMEM slot of 256 columns), 8 builds the tile's column
-// bitmap and streams Q and K, 9 streams V, 10 issues the MMAs.  A missing
-// block of a partial chunk is fetched at a row coordinate past the end of the
-// tensor, which TMA fills with zeros.
+// A CTA runs NWG independent pipelines.  Each has a softmax warpgroup (whose
+// thread 0 also issues that pipeline's MMAs) and two copy warps: one builds
+// the tile's column bitmap and gathers Q and the K chunks, the other gathers
+// the V chunks.  The copies are 16-byte cp.async transfers written straight
+// into the 128-byte-swizzled layout the MMA reads (many small copies in
+// flight reach a far higher gather rate than bulk tensor copies issued from
+// one thread, which are serviced one after another); a missing block of a
+// partial chunk is zero-filled.  Completion is signalled per stage with
+// cp.async.mbarrier.arrive.noinc, and the MMA-issuing thread fences the
+// generic-proxy writes after its barrier wait.  The copy warps never fence
+// (a proxy fence waits for the issuing thread's own copies in flight), and
+// the threads that fence never have copies in flight.  The copy warps give up
+// registers (setmaxnreg) to the softmax warpgroups.
 #pragma once
 
 #include "bsa_common.cuh"
@@ -38,46 +46,61 @@
 namespace bsa {
 namespace keys {
 
-constexpr int kThreads = 352;
-constexpr int kChunksResident = 7;        // S^T chunks held in one TMEM slot
-constexpr uint32_t kSlotCols = 256;
-constexpr uint32_t kOCol = 224;           // O^T columns inside a slot
+constexpr float kLazyMaxSlack = 8.0f;  // log2 units: P may reach 2^8 before a rescale
 
 template <int D>
 struct Cfg {
-  static constexpr int KATOMS = D / 64;
-  static constexpr int Q_BYTES = 32 * D * 2;      // one slot's Q: 32 rows
-  static constexpr int QATOM = 32 * 128;          // 32 rows x 128 B
-  static constexpr int CH_BYTES = 128 * D * 2;    // one K or V chunk: 128 key rows
-  static constexpr int CHATOM = 128 * 128;        // 128 rows x 128 B
-  static constexpr int NK = (D == 64) ? 3 : 2;   // K chunk ring
-  static constexpr int NV = (D == 64) ? 3 : 2;   // V chunk ring
-  static constexpr int NP = 4;                    // P^T buffers per slot
-  static constexpr int P_BYTES = 128 * 32 * 2;    // 128 keys x 32 queries, bf16
-  static constexpr bool PAD_A = (D == 64);        // zero upper half of the O^T A operand
+  static constexpr int NWG = (D == 64) ? 2 : 1;  // independent pipelines per CTA
+  static constexpr int THREADS = 128 * NWG + 128;  // + one warpgroup of copy warps
+  static constexpr int COPY_WG = NWG;            // warpgroup index of the copy warps
+  static constexpr int Q_BYTES = 32 * D * 2;     // 32 query rows
+  static constexpr int QATOM = 32 * 128;         // 32 rows x 128 B
+  static constexpr int CH_BYTES = 128 * D * 2;   // one K or V chunk: 128 key rows
+  static constexpr int CHATOM = 128 * 128;       // 128 rows x 128 B
+  static constexpr int NKS = 3;                  // K stages per pipeline
+  static constexpr int NVS = 2;                  // V stages per pipeline
+  static constexpr int P_BYTES = 128 * 32 * 2;   // P^T of a chunk: 128 keys x 32 queries
+  static constexpr bool PAD_A = (D == 64);       // zero upper half of the O^T A operand
+  // per-pipeline layout (offsets from the pipeline's base)
   static constexpr int OFF_Q = 0;
-  static constexpr int OFF_K = OFF_Q + 2 * Q_BYTES;
-  static constexpr int OFF_V = OFF_K + NK * CH_BYTES;
-  static constexpr int OFF_PAD = OFF_V + NV * CH_BYTES;
-  static constexpr int OFF_P = OFF_PAD + (PAD_A ? CHATOM : 0);
-  static constexpr int OFF_CTRL = OFF_P + 2 * NP * P_BYTES;
-  static_assert(Q_BYTES % 1024 == 0 && CH_BYTES % 1024 == 0 && P_BYTES % 1024 == 0, "alignment");
+  static constexpr int OFF_K = OFF_Q + Q_BYTES;
+  static constexpr int OFF_V = OFF_K + NKS * CH_BYTES;
+  static constexpr int OFF_P = OFF_V + NVS * CH_BYTES;
+  static constexpr int WG_BYTES = OFF_P + 2 * P_BYTES;
+  // CTA layout
+  static constexpr int OFF_PAD = NWG * WG_BYTES;
+  static constexpr int OFF_CTRL = OFF_PAD + (PAD_A ? CHATOM : 0);
+  static constexpr uint32_t TMEM_COLS = 128 * NWG;  // per pipeline: 2 S^T chunks + O^T
+  // register split: the copy warpgroup shrinks, the softmax warpgroups grow
+  static constexpr int REGS_AT_LAUNCH = 65536 / THREADS / 8 * 8;
+  static constexpr int REGS_COPY = 80;
+  static constexpr int REGS_SOFTMAX =
+      ((REGS_AT_LAUNCH * THREADS - REGS_COPY * 128) / (128 * NWG)) / 8 * 8 > 240
+          ? 240
+          : ((REGS_AT_LAUNCH * THREADS - REGS_COPY * 128) / (128 * NWG)) / 8 * 8;
+  static_assert(REGS_SOFTMAX * 128 * NWG + REGS_COPY * 128 <= REGS_AT_LAUNCH * THREADS,
+                "register split exceeds the launch's registers");
+  static_assert(Q_BYTES % 1024 == 0 && CH_BYTES % 1024 == 0 && WG_BYTES % 1024 == 0, "alignment");
+};
+
+struct alignas(16) PipeCtrl {
+  uint64_t bm_full[2], bm_empty[2];  // column bitmap written / read by all its readers
+  uint64_t qfull, qempty;            // Q copied (32 arrivals) / last QK of the tile done
+  uint64_t kfull[3], kempty[3];      // K stage copied (32 arrivals) / its QK done
+  uint64_t vfull[2], vempty[2];      // V stage copied (32 arrivals) / its PV done
+  uint64_t sbar[2];                  // S^T chunk ready (tcgen05.commit)
+  uint64_t obar;                     // one PV product completed (tcgen05.commit)
+  uint64_t fbar;                     // every MMA of this pipeline completed (teardown)
+  uint32_t bitmap[2][kMaxBitmapWords];
+  alignas(16) float red[4][32];
+  alignas(16) float bcast[32];  // read back as float4
+  alignas(16) float lsum[32];   // read back as float4
 };
 
 struct Ctrl {
-  uint64_t bm_full[2], bm_empty[2];
-  uint64_t q_full[2], q_empty[2];
-  uint64_t k_full[4], k_empty[4], v_full[4], v_empty[4];
-  uint64_t s_full[2], s_free[2];
-  uint64_t p_full[2][4], p_empty[2][4];
-  uint64_t pv_done[2], o_free[2];
-  uint64_t final_bar;
+  PipeCtrl pipe[2];
   uint32_t tmem_base;
   AbortFlag abort;
-  uint32_t bitmap[2][kMaxBitmapWords];
-  float red[2][4][32];
-  float bcast[2][32];
-  float lsum[2][32];
 };
 
 // Lane L ends with op over the 32 lanes of v[L] (v is consumed).
@@ -98,18 +121,89 @@ __device__ __forceinline__ float transpose_reduce(float (&v)[32], Op op) {
   return v[0];
 }
 
-struct TileInfo {
-  long long bh;
-  int r, h, L;
+// OR of `pred` over the 128 threads that meet at named barrier `id` (warp
+// reconverged first; non-aligned form, as for named_bar).
+__device__ __forceinline__ bool named_bar_or(int id, bool pred) {
+  __syncwarp();
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 q, %1, 0;\n\t"
+      "barrier.red.or.pred p, %2, 128, q;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(r)
+      : "r"(pred ? 1u : 0u), "r"(id)
+      : "memory");
+  return r != 0;
+}
+
+__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+
+template <int N>
+__device__ __forceinline__ void setmaxnreg_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void setmaxnreg_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
+// One copy warp gathers a chunk (4 blocks of 32 rows) into `stage` with the
+// 128-byte swizzle: 16-byte piece p of row r of an atom sits at piece
+// p ^ (r & 7).  Lane l copies piece l % PPR of rows l / PPR + k * (32 / PPR),
+// so a warp instruction moves 512 contiguous bytes and, per lane, the source
+// and destination of consecutive copies are a fixed stride apart; the swizzle
+// term repeats every 8 rows, so its few distinct values are precomputed once
+// per lane (GatherPlan).  blocks[b] < 0 marks a missing block (zero-filled).
+template <int D>
+struct GatherPlan {
+  static constexpr int PPR = D / 8;             // 16-byte pieces per row
+  static constexpr int RPI = 32 / PPR;          // rows covered by one warp instruction
+  static constexpr int ITERS = 32 / RPI;        // instructions per block
+  static constexpr int NSW = 8 / RPI;           // distinct (row & 7) patterns across iterations
+  int src;                                      // element offset of this lane's first piece
+  uint32_t dst[NSW];                            // byte offset inside a block, iteration i % NSW
+  __device__ __forceinline__ explicit GatherPlan(int lane) {
+    const int r0 = lane / PPR, pc = lane % PPR;
+    src = r0 * D + pc * 8;
+#pragma unroll
+    for (int v = 0; v < NSW; ++v) {
+      const int r = v * RPI + r0;               // row of iteration v (mod 8)
+      dst[v] = (pc >> 3) * (128 * 128) + r * 128 + (((pc & 7) ^ (r & 7)) << 4);
+    }
+  }
 };
 
-__device__ __forceinline__ TileInfo tile_info(const FwdArgs& a, long long tile) {
-  TileInfo ti;
-  ti.bh = tile / a.M;
-  ti.r = static_cast<int>(tile - ti.bh * a.M);
-  ti.h = static_cast<int>(ti.bh % a.H);
-  ti.L = 0;
-  return ti;
+template <int D>
+__device__ __forceinline__ void gather_chunk(uint32_t stage, const __nv_bfloat16* head,
+                                             const int (&blocks)[4], const GatherPlan<D>& g) {
+  using G = GatherPlan<D>;
+#pragma unroll
+  for (int b = 0; b < 4; ++b) {
+    const int j = blocks[b];
+    const uint32_t bytes = j >= 0 ? 16u : 0u;
+    const __nv_bfloat16* src = head + static_cast<long long>(j >= 0 ? j : 0) * 32 * D + g.src;
+    const uint32_t dst = stage + b * 4096;
+#pragma unroll
+    for (int i = 0; i < G::ITERS; ++i)
+      cp_async_16(dst + (i / G::NSW) * (8 * 128) + g.dst[i % G::NSW], src + i * G::RPI * D, bytes);
+  }
+}
+
+struct TileRef {
+  long long bh;
+  int r, h;
+};
+
+__device__ __forceinline__ TileRef tile_ref(const FwdArgs& a, long long tile) {
+  TileRef t;
+  t.bh = tile / a.M;
+  t.r = static_cast<int>(tile - t.bh * a.M);
+  t.h = static_cast<int>(t.bh % a.H);
+  return t;
 }
 
 __device__ __forceinline__ int popcount_words(const uint32_t* w, int W) {
@@ -118,30 +212,31 @@ __device__ __forceinline__ int popcount_words(const uint32_t* w, int W) {
   return n;
 }
 
-// ------------------------------------------------------- Q / K producer warp
+// ------------------------------------------------------------ copy warps
+// K warp: builds each tile's column bitmap, then gathers Q and the K chunks.
 template <int D>
-__device__ void producer_qk(const CUtensorMap* tmQ, const CUtensorMap* tmK, const FwdArgs& a,
-                            uint8_t* smem, Ctrl* ctl) {
+__device__ void copy_warp_qk(const FwdArgs& a, uint8_t* base, PipeCtrl* pc, AbortFlag* ab, int wg) {
   using C = Cfg<D>;
   const int lane = threadIdx.x & 31;
-  uint32_t k_loads = 0, q_loads[2] = {0, 0};
+  const uint32_t q_s = smem_u32(base + C::OFF_Q);
+  const uint32_t k_s = smem_u32(base + C::OFF_K);
+  const GatherPlan<D> plan(lane);
+  uint32_t k_issued = 0, q_issued = 0;
   bool ok = true;
-  if (lane == 0) {
-    prefetch_tensormap(tmQ);
-    prefetch_tensormap(tmK);
-  }
+  const long long stride = static_cast<long long>(gridDim.x) * C::NWG;
   int k = 0;
-  for (long long tile = blockIdx.x; tile < a.num_tiles; tile += gridDim.x, ++k) {
+  for (long long tile = static_cast<long long>(blockIdx.x) * C::NWG + wg; ok && tile < a.num_tiles;
+       tile += stride, ++k) {
     const int slot = k & 1;
     int w_ok = 1;
-    if (lane == 0) w_ok = wait_bounded(&ctl->bm_empty[slot], ((k >> 1) & 1) ^ 1, &ctl->abort);
+    if (lane == 0) w_ok = wait_bounded(&pc->bm_empty[slot], ((k >> 1) & 1) ^ 1, ab);
     if (!__shfl_sync(0xffffffffu, w_ok, 0)) { ok = false; break; }
-    uint32_t* bm = ctl->bitmap[slot];
+    uint32_t* bm = pc->bitmap[slot];
     for (int w = lane; w < a.W; w += 32) bm[w] = 0u;
     __syncwarp();
-    const TileInfo ti = tile_info(a, tile);
-    const int beg = __ldg(a.row_ptr + (static_cast<long long>(ti.h) * a.M + ti.r));
-    const int end = __ldg(a.row_ptr + (static_cast<long long>(ti.h) * a.M + ti.r + 1));
+    const TileRef t = tile_ref(a, tile);
+    const int beg = __ldg(a.row_ptr + (static_cast<long long>(t.h) * a.M + t.r));
+    const int end = __ldg(a.row_ptr + (static_cast<long long>(t.h) * a.M + t.r + 1));
     if (end < beg) {
       if (lane == 0) atomicOr(&g_status, BSA_STATUS_BAD_ROW_PTR);
     } else {
@@ -151,471 +246,407 @@ __device__ void producer_qk(const CUtensorMap* tmQ, const CUtensorMap* tmK, cons
           atomicOr(&g_status, BSA_STATUS_BAD_COLUMN);
           continue;
         }
-        if (a.causal && j > ti.r) continue;  // wholly above the diagonal: no allowed key
+        if (a.causal && j > t.r) continue;  // wholly above the diagonal: no allowed key
         atomicOr(&bm[j >> 5], 1u << (j & 31));
       }
     }
     __threadfence_block();
     __syncwarp();
-    if (lane == 0) {
-      mbar_arrive(&ctl->bm_full[slot]);
-      const int L = popcount_words(bm, a.W);
-      if (L > 0) {
-        ok = wait_bounded(&ctl->q_empty[slot], (q_loads[slot] & 1) ^ 1, &ctl->abort);
-        if (ok) {
-          mbar_arrive_expect_tx(&ctl->q_full[slot], C::Q_BYTES);
-          for (int ka = 0; ka < C::KATOMS; ++ka)
-            tma_load_3d(smem + C::OFF_Q + slot * C::Q_BYTES + ka * C::QATOM, tmQ,
-                        &ctl->q_full[slot], ka * 64, ti.r * 32, static_cast<int>(ti.bh));
-          ++q_loads[slot];
-        }
-        BitIter it(bm, a.W);
-        const int nch = (L + 3) / 4;
-        for (int c = 0; ok && c < nch; ++c) {
-          const uint32_t ks = k_loads % C::NK;
-          ok = wait_bounded(&ctl->k_empty[ks], ((k_loads / C::NK) & 1) ^ 1, &ctl->abort);
-          if (!ok) break;
-          mbar_arrive_expect_tx(&ctl->k_full[ks], C::CH_BYTES);
-          for (int b = 0; b < 4; ++b) {
-            const int j = it.next();
-            const int row = j >= 0 ? j * 32 : a.N;  // past the end: zero-filled by TMA
-            for (int ka = 0; ka < C::KATOMS; ++ka)
-              tma_load_3d(smem + C::OFF_K + ks * C::CH_BYTES + ka * C::CHATOM + b * 4096, tmK,
-                          &ctl->k_full[ks], ka * 64, row, static_cast<int>(ti.bh));
-          }
-          ++k_loads;
-        }
+    if (lane == 0) mbar_arrive(&pc->bm_full[slot]);
+    const int L = popcount_words(bm, a.W);
+    if (L == 0) continue;
+    const __nv_bfloat16* khead = a.K + t.bh * static_cast<long long>(a.N) * D;
+    // Q: 32 rows, 128-byte swizzle
+    if (lane == 0) w_ok = wait_bounded(&pc->qempty, (q_issued & 1) ^ 1, ab);
+    if (!__shfl_sync(0xffffffffu, w_ok, 0)) { ok = false; break; }
+    {
+      const __nv_bfloat16* qsrc = a.Q + (t.bh * a.N + static_cast<long long>(t.r) * 32) * D;
+      for (int p = lane; p < 32 * D / 8; p += 32) {
+        const int rr = p / (D / 8), pp = p % (D / 8);
+        cp_async_16(q_s + (pp >> 3) * C::QATOM + rr * 128 + (((pp & 7) ^ (rr & 7)) << 4),
+                    qsrc + rr * D + pp * 8, 16u);
       }
+      cp_async_arrive_noinc(&pc->qfull);
+      ++q_issued;
     }
-    if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) { ok = false; break; }
+    BitIter it(bm, a.W);
+    const int nch = (L + 3) / 4;
+    for (int c = 0; c < nch; ++c) {
+      int blk[4];
+      for (int b = 0; b < 4; ++b) blk[b] = it.next();
+      const uint32_t s = k_issued % C::NKS;
+      if (lane == 0) w_ok = wait_bounded(&pc->kempty[s], ((k_issued / C::NKS) & 1) ^ 1, ab);
+      if (!__shfl_sync(0xffffffffu, w_ok, 0)) { ok = false; break; }
+      gather_chunk<D>(k_s + s * C::CH_BYTES, khead, blk, plan);
+      cp_async_arrive_noinc(&pc->kfull[s]);
+      ++k_issued;
+    }
   }
-  if (!ok && lane == 0) {
-    for (int s = 0; s < 2; ++s)
-      if (q_loads[s] > 0) wait_drain(&ctl->q_full[s], (q_loads[s] - 1) & 1);
-    for (uint32_t s = 0; s < static_cast<uint32_t>(C::NK); ++s)
-      if (k_loads > s) {
-        const uint32_t last = s + C::NK * ((k_loads - 1 - s) / C::NK);
-        wait_drain(&ctl->k_full[s], (last / C::NK) & 1);
-      }
-  }
+  cp_async_wait<0>();
   __syncwarp();
 }
 
-// --------------------------------------------------------------- V producer
+// V warp: gathers the V chunks of each tile.
 template <int D>
-__device__ void producer_v(const CUtensorMap* tmV, const FwdArgs& a, uint8_t* smem, Ctrl* ctl) {
+__device__ void copy_warp_v(const FwdArgs& a, uint8_t* base, PipeCtrl* pc, AbortFlag* ab, int wg) {
   using C = Cfg<D>;
   const int lane = threadIdx.x & 31;
-  uint32_t v_loads = 0;
+  const uint32_t v_s = smem_u32(base + C::OFF_V);
+  const GatherPlan<D> plan(lane);
+  uint32_t v_issued = 0;
   bool ok = true;
-  if (lane == 0) {
-    prefetch_tensormap(tmV);
-    int k = 0;
-    for (long long tile = blockIdx.x; ok && tile < a.num_tiles; tile += gridDim.x, ++k) {
-      const int slot = k & 1;
-      if (!wait_bounded(&ctl->bm_full[slot], (k >> 1) & 1, &ctl->abort)) { ok = false; break; }
-      const TileInfo ti = tile_info(a, tile);
-      const uint32_t* bm = ctl->bitmap[slot];
-      const int L = popcount_words(bm, a.W);
-      BitIter it(bm, a.W);
-      const int nch = (L + 3) / 4;
-      for (int c = 0; c < nch; ++c) {
-        const uint32_t vs = v_loads % C::NV;
-        ok = wait_bounded(&ctl->v_empty[vs], ((v_loads / C::NV) & 1) ^ 1, &ctl->abort);
-        if (!ok) break;
-        mbar_arrive_expect_tx(&ctl->v_full[vs], C::CH_BYTES);
-        for (int b = 0; b < 4; ++b) {
-          const int j = it.next();
-          const int row = j >= 0 ? j * 32 : a.N;
-          for (int ka = 0; ka < C::KATOMS; ++ka)
-            tma_load_3d(smem + C::OFF_V + vs * C::CH_BYTES + ka * C::CHATOM + b * 4096, tmV,
-                        &ctl->v_full[vs], ka * 64, row, static_cast<int>(ti.bh));
-        }
-        ++v_loads;
-      }
-      mbar_arrive(&ctl->bm_empty[slot]);
+  const long long stride = static_cast<long long>(gridDim.x) * C::NWG;
+  int k = 0;
+  for (long long tile = static_cast<long long>(blockIdx.x) * C::NWG + wg; ok && tile < a.num_tiles;
+       tile += stride, ++k) {
+    const int slot = k & 1;
+    int w_ok = 1;
+    if (lane == 0) w_ok = wait_bounded(&pc->bm_full[slot], (k >> 1) & 1, ab);
+    if (!__shfl_sync(0xffffffffu, w_ok, 0)) { ok = false; break; }
+    const uint32_t* bm = pc->bitmap[slot];
+    const TileRef t = tile_ref(a, tile);
+    const __nv_bfloat16* vhead = a.V + t.bh * static_cast<long long>(a.N) * D;
+    const int nch = (popcount_words(bm, a.W) + 3) / 4;
+    BitIter it(bm, a.W);
+    for (int c = 0; c < nch; ++c) {
+      int blk[4];
+      for (int b = 0; b < 4; ++b) blk[b] = it.next();
+      const uint32_t s = v_issued % C::NVS;
+      if (lane == 0) w_ok = wait_bounded(&pc->vempty[s], ((v_issued / C::NVS) & 1) ^ 1, ab);
+      if (!__shfl_sync(0xffffffffu, w_ok, 0)) { ok = false; break; }
+      gather_chunk<D>(v_s + s * C::CH_BYTES, vhead, blk, plan);
+      cp_async_arrive_noinc(&pc->vfull[s]);
+      ++v_issued;
     }
-    if (!ok)
-      for (uint32_t s = 0; s < static_cast<uint32_t>(C::NV); ++s)
-        if (v_loads > s) {
-          const uint32_t last = s + C::NV * ((v_loads - 1 - s) / C::NV);
-          wait_drain(&ctl->v_full[s], (last / C::NV) & 1);
-        }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&pc->bm_empty[slot]);
   }
+  cp_async_wait<0>();
   __syncwarp();
 }
 
-// ------------------------------------------------------------------ MMA warp
-struct Item {
-  int k;        // CTA-local tile index
-  int slot;
-  int c0, nc;   // first chunk of the group and its chunk count
-  bool first, last;
-};
-
+// ------------------------------------------------------- softmax warpgroup
 template <int D>
-struct MmaState {
-  uint32_t k_cons = 0, v_cons = 0;
-  uint32_t q_uses[2] = {0, 0}, s_uses[2] = {0, 0}, chunks[2] = {0, 0}, o_uses[2] = {0, 0};
-};
-
-template <int D>
-__device__ bool issue_qk(const Item& X, MmaState<D>& st, uint8_t* smem, Ctrl* ctl, uint32_t tmem) {
+__device__ void softmax_wg(const FwdArgs& a, uint8_t* smem, Ctrl* ctl, uint32_t tmem_base, int wg) {
   using C = Cfg<D>;
-  constexpr uint32_t kIdesc = idesc_bf16_f32(128, 32, false, false);
-  const int s = X.slot;
-  if (X.first) {
-    if (!wait_bounded(&ctl->q_full[s], st.q_uses[s] & 1, &ctl->abort)) return false;
-    ++st.q_uses[s];
-  }
-  if (!wait_bounded(&ctl->s_free[s], (st.s_uses[s] & 1) ^ 1, &ctl->abort)) return false;
-  ++st.s_uses[s];
-  const uint32_t q_base = smem_u32(smem + C::OFF_Q + s * C::Q_BYTES);
-  const uint32_t k_base = smem_u32(smem + C::OFF_K);
-  for (int c = 0; c < X.nc; ++c) {
-    const uint32_t ks = st.k_cons % C::NK;
-    if (!wait_bounded(&ctl->k_full[ks], (st.k_cons / C::NK) & 1, &ctl->abort)) return false;
-    tc_fence_after();
-#pragma unroll
-    for (int kk = 0; kk < D / 16; ++kk) {
-      const uint64_t ad = sdesc_sw128(k_base + ks * C::CH_BYTES + (kk >> 2) * C::CHATOM + (kk & 3) * 32,
-                                      16, 1024);
-      const uint64_t bd = sdesc_sw128(q_base + (kk >> 2) * C::QATOM + (kk & 3) * 32, 16, 1024);
-      umma_bf16_ss(tmem + s * kSlotCols + c * 32, ad, bd, kIdesc, kk > 0 ? 1u : 0u);
-    }
-    umma_commit(&ctl->k_empty[ks]);
-    ++st.k_cons;
-  }
-  umma_commit(&ctl->s_full[s]);
-  if (X.last) umma_commit(&ctl->q_empty[s]);
-  return true;
-}
-
-template <int D>
-__device__ bool issue_pv(const Item& X, MmaState<D>& st, uint8_t* smem, Ctrl* ctl, uint32_t tmem) {
-  using C = Cfg<D>;
-  // A = V^T (MN-major, 128-byte swizzle), B = P^T (MN-major, 64-byte swizzle).
-  constexpr uint32_t kIdesc = idesc_bf16_f32(128, 32, true, true);
-  const int s = X.slot;
-  if (X.first) {
-    if (!wait_bounded(&ctl->o_free[s], (st.o_uses[s] & 1) ^ 1, &ctl->abort)) return false;
-    ++st.o_uses[s];
-  }
-  const uint32_t v_base = smem_u32(smem + C::OFF_V);
-  const uint32_t pad = smem_u32(smem + C::OFF_PAD);
-  const uint32_t p_base = smem_u32(smem + C::OFF_P + s * C::NP * C::P_BYTES);
-  for (int c = 0; c < X.nc; ++c) {
-    const uint32_t g = st.chunks[s];
-    const uint32_t pb = g % C::NP;
-    if (!wait_bounded(&ctl->p_full[s][pb], (g / C::NP) & 1, &ctl->abort)) return false;
-    const uint32_t vs = st.v_cons % C::NV;
-    if (!wait_bounded(&ctl->v_full[vs], (st.v_cons / C::NV) & 1, &ctl->abort)) return false;
-    tc_fence_after();
-    const uint32_t vstage = v_base + vs * C::CH_BYTES;
-    const uint32_t lbo = C::PAD_A ? (pad - vstage) : static_cast<uint32_t>(C::CHATOM);
-#pragma unroll
-    for (int kk = 0; kk < 8; ++kk) {  // 128 keys, 16 per MMA
-      const uint64_t ad = sdesc(vstage + kk * 2048, lbo, 1024, kLayoutSW128);
-      const uint64_t bd = sdesc(p_base + pb * C::P_BYTES + kk * 1024, C::P_BYTES, 512, kLayoutSW64);
-      umma_bf16_ss(tmem + s * kSlotCols + kOCol, ad, bd, kIdesc,
-                   (X.first && c == 0 && kk == 0) ? 0u : 1u);
-    }
-    umma_commit(&ctl->v_empty[vs]);
-    umma_commit(&ctl->p_empty[s][pb]);
-    ++st.v_cons;
-    ++st.chunks[s];
-  }
-  umma_commit(&ctl->pv_done[s]);
-  return true;
-}
-
-template <int D>
-__device__ void mma_role(const FwdArgs& a, uint8_t* smem, Ctrl* ctl, uint32_t tmem) {
-  MmaState<D> st;
-  Item pending{};
-  bool has_pending = false;
-  bool ok = true;
-  int k = 0;
-  for (long long tile = blockIdx.x; ok && tile < a.num_tiles; tile += gridDim.x, ++k) {
-    const int slot = k & 1;
-    if (!wait_bounded(&ctl->bm_full[slot], (k >> 1) & 1, &ctl->abort)) { ok = false; break; }
-    const int L = popcount_words(ctl->bitmap[slot], a.W);
-    mbar_arrive(&ctl->bm_empty[slot]);
-    if (L == 0) continue;
-    const int nch = (L + 3) / 4;
-    for (int c0 = 0; ok && c0 < nch; c0 += kChunksResident) {
-      Item X;
-      X.k = k;
-      X.slot = slot;
-      X.c0 = c0;
-      X.nc = min(kChunksResident, nch - c0);
-      X.first = (c0 == 0);
-      X.last = (c0 + kChunksResident >= nch);
-      // QK of a new tile goes ahead of the PV of the previous tile, so one
-      // warpgroup's softmax overlaps the other's tensor-core work; within a
-      // tile the next group's QK waits for this group's PV.
-      if (has_pending && pending.k == k) {
-        ok = issue_pv<D>(pending, st, smem, ctl, tmem) && issue_qk<D>(X, st, smem, ctl, tmem);
-      } else {
-        ok = issue_qk<D>(X, st, smem, ctl, tmem);
-        if (ok && has_pending) ok = issue_pv<D>(pending, st, smem, ctl, tmem);
-      }
-      pending = X;
-      has_pending = true;
-    }
-  }
-  if (ok && has_pending) issue_pv<D>(pending, st, smem, ctl, tmem);
-  umma_commit(&ctl->final_bar);
-  wait_drain(&ctl->final_bar, 0);
-}
-
-// --------------------------------------------------------- softmax warpgroups
-template <int D>
-__device__ void softmax_role(const FwdArgs& a, uint8_t* smem, Ctrl* ctl, uint32_t tmem, int wg) {
-  using C = Cfg<D>;
+  constexpr float kNegInf = -INFINITY;
+  constexpr uint32_t kIdescQK = idesc_bf16_f32(128, 32, false, false);  // K, Q: K-major
+  constexpr uint32_t kIdescPV = idesc_bf16_f32(128, 32, true, true);    // V^T, P^T: MN-major
+  PipeCtrl* pc = &ctl->pipe[wg];
+  AbortFlag* ab = &ctl->abort;
   const int tid = threadIdx.x & 127;
   const int warp = tid >> 5;
   const int lane = tid & 31;
-  const int slot = wg;
+  const int bar_id = 1 + wg;
+  uint8_t* base = smem + wg * C::WG_BYTES;
+  const uint32_t q_s = smem_u32(base + C::OFF_Q);
+  const uint32_t k_s = smem_u32(base + C::OFF_K);
+  const uint32_t v_s = smem_u32(base + C::OFF_V);
+  const uint32_t p_s = smem_u32(base + C::OFF_P);
+  const uint32_t pad_s = smem_u32(smem + C::OFF_PAD);
+  const uint32_t tmem = tmem_base + wg * 128;
   const uint32_t t_lane = static_cast<uint32_t>(warp * 32) << 16;
-  const uint32_t s_col = tmem + slot * kSlotCols + t_lane;
-  const uint32_t o_col = tmem + slot * kSlotCols + kOCol + t_lane;
-  const uint32_t p_row0 = smem_u32(smem + C::OFF_P + slot * C::NP * C::P_BYTES) + tid * 64;
-  const int bar_id = 1 + slot;
-  constexpr float kNegInf = -INFINITY;
-  uint32_t s_uses = 0, chunks = 0, pv_waits = 0;
+  const uint32_t s_col = tmem + t_lane;       // S^T chunk buffers at +0 and +32
+  const uint32_t o_col = tmem + 64 + t_lane;  // O^T
+  const float scale_log2 = a.scale_log2;
+  const int causal = a.causal;
+  const int W = a.W, N = a.N;
 
-  for (int k = wg;; k += 2) {
-    const long long tile = blockIdx.x + static_cast<long long>(k) * gridDim.x;
-    if (tile >= a.num_tiles) break;
-    if (!warp_wait(&ctl->bm_full[slot], (k >> 1) & 1, &ctl->abort)) return;
-    const uint32_t* bm = ctl->bitmap[slot];
-    const TileInfo ti = tile_info(a, tile);
-    const int L = popcount_words(bm, a.W);
+  // running counters: barrier phases continue across tiles
+  uint32_t k_used = 0, v_used = 0, q_used = 0;
+  uint32_t s_uses[2] = {0, 0};
+  uint32_t pv_issued = 0, pv_seen = 0;
+  bool ok = true;
+
+  // all 128 threads agree: true iff every one of them passes `mine`
+  auto all_ok = [&](bool mine) { return !named_bar_or(bar_id, !mine); };
+  // The first `count` PVs of this pipeline completed.  Callers keep `count`
+  // within one of the PVs issued: obar is one barrier whose phases are told
+  // apart by parity, so at most one of its completions may go unobserved.
+  auto ensure_pv_done = [&](uint32_t count) -> bool {
+    bool good = true;
+    while (good && pv_seen < count) {
+      good = wait_bounded(&pc->obar, pv_seen & 1, ab);
+      ++pv_seen;
+    }
+    return good;
+  };
+  // thread 0: S^T[sb] = K Q^T for the next K chunk
+  auto issue_qk = [&](int sb, bool last) -> bool {
+    const uint32_t ks = k_used % C::NKS;
+    if (!wait_bounded(&pc->kfull[ks], (k_used / C::NKS) & 1, ab)) return false;
+    fence_proxy_async_smem();  // the copy warp's writes, seen through the barrier
+    tc_fence_after();
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+      const uint64_t ad =
+          sdesc_sw128(k_s + ks * C::CH_BYTES + (kk >> 2) * C::CHATOM + (kk & 3) * 32, 16, 1024);
+      const uint64_t bd = sdesc_sw128(q_s + (kk >> 2) * C::QATOM + (kk & 3) * 32, 16, 1024);
+      umma_bf16_ss(tmem + sb * 32, ad, bd, kIdescQK, kk > 0 ? 1u : 0u);
+    }
+    umma_commit(&pc->kempty[ks]);
+    umma_commit(&pc->sbar[sb]);
+    if (last) umma_commit(&pc->qempty);
+    return true;
+  };
+
+  const long long stride = static_cast<long long>(gridDim.x) * C::NWG;
+  int k = 0;
+  for (long long tile = static_cast<long long>(blockIdx.x) * C::NWG + wg; ok && tile < a.num_tiles;
+       tile += stride, ++k) {
+    const int slot = k & 1;
+    const TileRef t = tile_ref(a, tile);
+    // ---- the tile's columns
+    if (!(ok = all_ok(wait_bounded(&pc->bm_full[slot], (k >> 1) & 1, ab)))) break;
+    const uint32_t* bm = pc->bitmap[slot];
+    const int L = popcount_words(bm, W);
     int diag_pos = -1;
-    if (a.causal && ((bm[ti.r >> 5] >> (ti.r & 31)) & 1u)) {
+    if (causal && ((bm[t.r >> 5] >> (t.r & 31)) & 1u)) {
       diag_pos = 0;
-      for (int w = 0; w < (ti.r >> 5); ++w) diag_pos += __popc(bm[w]);
-      diag_pos += __popc(bm[ti.r >> 5] & ((1u << (ti.r & 31)) - 1u));
+      for (int w = 0; w < (t.r >> 5); ++w) diag_pos += __popc(bm[w]);
+      diag_pos += __popc(bm[t.r >> 5] & ((1u << (t.r & 31)) - 1u));
     }
     __syncwarp();
-    if (lane == 0) mbar_arrive(&ctl->bm_empty[slot]);
-    const long long row0 = ti.bh * a.N + static_cast<long long>(ti.r) * 32;  // first query row
-
+    if (lane == 0) mbar_arrive(&pc->bm_empty[slot]);
+    const long long row0 = t.bh * N + static_cast<long long>(t.r) * 32;  // first query row
     if (L == 0) {  // no key at all: O = 0, LSE = -inf
       uint4* o = reinterpret_cast<uint4*>(a.O + row0 * D);
       for (int i = tid; i < 32 * D / 8; i += 128) o[i] = make_uint4(0u, 0u, 0u, 0u);
       if (warp == 0) a.LSE[row0 + lane] = kNegInf;
       continue;
     }
-
     const int nch = (L + 3) / 4;
-    float mu[32];     // running max per query (log2 units), -inf replaced by 0
+
+    bool mine = true;
+    if (tid == 0) {
+      mine = wait_bounded(&pc->qfull, q_used & 1, ab) && issue_qk(0, nch == 1);
+    }
+    ++q_used;
+    ++k_used;
+
+    float mu[32];     // running max per query (log2 units of the scaled score)
     float lpart[32];  // this thread's partial row sums
-    float m_own = kNegInf;  // running max of query `lane`, -inf kept
+    float m_own = kNegInf;  // running max of query `lane`
 #pragma unroll
     for (int q = 0; q < 32; ++q) {
-      mu[q] = 0.f;
+      mu[q] = kNegInf;
       lpart[q] = 0.f;
     }
-    for (int c0 = 0; c0 < nch; c0 += kChunksResident) {
-      const int nc = min(kChunksResident, nch - c0);
-      if (!warp_wait(&ctl->s_full[slot], s_uses & 1, &ctl->abort)) return;
-      ++s_uses;
+    const uint32_t pv_base = pv_issued;
+
+    for (int c = 0; c < nch; ++c) {
+      const int sb = c & 1;
+      // ---- S^T of chunk c ready; thread 0 starts QK of chunk c + 1 at once
+      mine = mine && wait_bounded(&pc->sbar[sb], s_uses[sb] & 1, ab);
+      ++s_uses[sb];
+      if (tid == 0 && mine && c + 1 < nch) mine = issue_qk(sb ^ 1, c + 2 == nch);
+      if (c + 1 < nch) ++k_used;
+      if (!(ok = all_ok(mine))) break;
       tc_fence_after();
 
-      // ---- pass 1: per-query maximum over the key rows of this group
-      float mx[32];
-#pragma unroll
-      for (int q = 0; q < 32; ++q) mx[q] = kNegInf;
-      for (int c = 0; c < nc; ++c) {
-        const int blk = 4 * (c0 + c) + warp;  // block slot held by this warp
-        if (blk < L) {
-          uint32_t u[32];
-          tmem_ld32(s_col + c * 32, u);
-          tmem_wait_ld();
-          if (blk == diag_pos) {
-#pragma unroll
-            for (int q = 0; q < 32; ++q) {
-              const float v = (lane > q) ? kNegInf : __uint_as_float(u[q]) * a.scale_log2;
-              mx[q] = fmaxf(mx[q], v);
-            }
-          } else {
-#pragma unroll
-            for (int q = 0; q < 32; ++q) mx[q] = fmaxf(mx[q], __uint_as_float(u[q]) * a.scale_log2);
-          }
-        }
-      }
-      const float wmax = transpose_reduce(mx, [](float x, float y) { return fmaxf(x, y); });
-      ctl->red[slot][warp][lane] = wmax;
-      named_bar(bar_id, 128);
-      const float gmax = fmaxf(fmaxf(ctl->red[slot][0][lane], ctl->red[slot][1][lane]),
-                               fmaxf(ctl->red[slot][2][lane], ctl->red[slot][3][lane]));
-      const float m_new_own = fmaxf(m_own, gmax);
-      if (warp == 0) ctl->bcast[slot][lane] = (m_new_own == kNegInf) ? 0.f : m_new_own;
-      named_bar(bar_id, 128);
-      m_own = m_new_own;
-      float mnew[32];
-#pragma unroll
-      for (int q = 0; q < 32; q += 4) {
-        const float4 t4 = *reinterpret_cast<const float4*>(&ctl->bcast[slot][q]);
-        mnew[q] = t4.x;
-        mnew[q + 1] = t4.y;
-        mnew[q + 2] = t4.z;
-        mnew[q + 3] = t4.w;
-      }
-
-      // ---- rescale what earlier groups of this row accumulated
-      if (c0 > 0) {
-        if (!warp_wait(&ctl->pv_done[slot], pv_waits & 1, &ctl->abort)) return;
-        ++pv_waits;
-        tc_fence_after();
+      // ---- scores of this thread's key row for the 32 queries
+      const int blk_slot = 4 * c + warp;  // block slot held by this warp
+      const bool valid = blk_slot < L;
+      const bool diag = (blk_slot == diag_pos);
+      float x[32];
+      if (valid) {
         uint32_t u[32];
-        tmem_ld32(o_col, u);
+        tmem_ld32(s_col + sb * 32, u);
         tmem_wait_ld();
 #pragma unroll
         for (int q = 0; q < 32; ++q) {
-          const float f = ex2_approx(mu[q] - mnew[q]);
-          u[q] = __float_as_uint(__uint_as_float(u[q]) * f);
-          lpart[q] *= f;
+          const float v = __uint_as_float(u[q]) * scale_log2;
+          x[q] = (diag && lane > q) ? kNegInf : v;
         }
-        tmem_st32(o_col, u);
-        tmem_wait_st();
-      }
+      } else {
 #pragma unroll
-      for (int q = 0; q < 32; ++q) mu[q] = mnew[q];
-
-      // ---- pass 2: P^T = 2^(s - max) in bf16, chunk by chunk
-      for (int c = 0; c < nc; ++c) {
-        const uint32_t pb = chunks % C::NP;
-        if (!warp_wait(&ctl->p_empty[slot][pb], ((chunks / C::NP) & 1) ^ 1, &ctl->abort)) return;
-        const int blk = 4 * (c0 + c) + warp;
-        if (blk < L) {
-          uint32_t u[32];
-          tmem_ld32(s_col + c * 32, u);
-          tmem_wait_ld();
-          const bool diag = (blk == diag_pos);
-          uint32_t pk[16];
-#pragma unroll
-          for (int q = 0; q < 32; q += 2) {
-            float x0 = __uint_as_float(u[q]) * a.scale_log2 - mu[q];
-            float x1 = __uint_as_float(u[q + 1]) * a.scale_log2 - mu[q + 1];
-            if (diag && lane > q) x0 = kNegInf;
-            if (diag && lane > q + 1) x1 = kNegInf;
-            const float p0 = ex2_approx(x0);
-            const float p1 = ex2_approx(x1);
-            lpart[q] += p0;
-            lpart[q + 1] += p1;
-            pk[q >> 1] = pack_bf16x2(p0, p1);
-          }
-          // row `tid` of P^T (64 bytes), 64-byte swizzle: chunk c sits at c ^ ((tid >> 1) & 3)
-          const uint32_t base = p_row0 + pb * C::P_BYTES;
-          const uint32_t sw = (tid >> 1) & 3;
-#pragma unroll
-          for (int c16 = 0; c16 < 4; ++c16)
-            st_shared_v4(base + ((c16 ^ sw) << 4), pk[4 * c16], pk[4 * c16 + 1], pk[4 * c16 + 2],
-                         pk[4 * c16 + 3]);
-        }
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&ctl->p_full[slot][pb]);
-        ++chunks;
+        for (int q = 0; q < 32; ++q) x[q] = kNegInf;
       }
       tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&ctl->s_free[slot]);
+
+      // ---- lazy maximum: exact update only when a score outgrows it by > 2^8
+      bool viol = false;
+#pragma unroll
+      for (int q = 0; q < 32; ++q) viol |= (x[q] > mu[q] + kLazyMaxSlack);
+      if (named_bar_or(bar_id, viol)) {
+        float mx[32];
+#pragma unroll
+        for (int q = 0; q < 32; ++q) mx[q] = x[q];
+        const float wmax = transpose_reduce(mx, [](float p, float s) { return fmaxf(p, s); });
+        pc->red[warp][lane] = wmax;
+        named_bar(bar_id, 128);
+        const float gmax = fmaxf(fmaxf(pc->red[0][lane], pc->red[1][lane]),
+                                 fmaxf(pc->red[2][lane], pc->red[3][lane]));
+        m_own = fmaxf(m_own, gmax);
+        if (warp == 0) pc->bcast[lane] = m_own;
+        named_bar(bar_id, 128);
+        float mnew[32];
+#pragma unroll
+        for (int q = 0; q < 32; q += 4) {
+          const float4 t4 = *reinterpret_cast<const float4*>(&pc->bcast[q]);
+          mnew[q] = t4.x;
+          mnew[q + 1] = t4.y;
+          mnew[q + 2] = t4.z;
+          mnew[q + 3] = t4.w;
+        }
+        if (c > 0) {  // rescale what the earlier chunks accumulated
+          if (!(ok = all_ok(ensure_pv_done(pv_base + c)))) break;
+          tc_fence_after();
+          uint32_t u[32];
+          tmem_ld32(o_col, u);
+          tmem_wait_ld();
+#pragma unroll
+          for (int q = 0; q < 32; ++q) {
+            const float f = (mu[q] == kNegInf) ? 0.f : ex2_approx(mu[q] - mnew[q]);
+            u[q] = __float_as_uint(__uint_as_float(u[q]) * f);
+            lpart[q] *= f;
+          }
+          tmem_st32(o_col, u);
+          tmem_wait_st();
+        }
+#pragma unroll
+        for (int q = 0; q < 32; ++q) mu[q] = mnew[q];
+      }
+
+      // ---- P^T = 2^(s - max) in bf16 into buffer sb.  PV(c - 1) is observed
+      // here every iteration (see ensure_pv_done); that also frees buffer sb,
+      // last read by PV(c - 2).
+      if (c >= 1 && !(ok = all_ok(ensure_pv_done(pv_base + c)))) break;
+      if (valid) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int q = 0; q < 32; q += 2) {
+          const float p0 = ex2_approx(x[q] - (mu[q] == kNegInf ? 0.f : mu[q]));
+          const float p1 = ex2_approx(x[q + 1] - (mu[q + 1] == kNegInf ? 0.f : mu[q + 1]));
+          lpart[q] += p0;
+          lpart[q + 1] += p1;
+          pk[q >> 1] = pack_bf16x2(p0, p1);
+        }
+        const uint32_t rowp = p_s + sb * C::P_BYTES + tid * 64;  // 64-byte swizzle
+        const uint32_t sw = (tid >> 1) & 3;
+#pragma unroll
+        for (int c16 = 0; c16 < 4; ++c16)
+          st_shared_v4(rowp + ((c16 ^ sw) << 4), pk[4 * c16], pk[4 * c16 + 1], pk[4 * c16 + 2],
+                       pk[4 * c16 + 3]);
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+
+      // ---- PV of chunk c (thread 0 issues after every P^T row is written)
+      named_bar(bar_id, 128);
+      mine = true;
+      if (tid == 0) {
+        const uint32_t vs = v_used % C::NVS;
+        mine = wait_bounded(&pc->vfull[vs], (v_used / C::NVS) & 1, ab);
+        if (mine) {
+          fence_proxy_async_smem();  // the copy warp's writes, seen through the barrier
+          tc_fence_after();
+          const uint32_t vstage = v_s + vs * C::CH_BYTES;
+          const uint32_t lbo = C::PAD_A ? (pad_s - vstage) : static_cast<uint32_t>(C::CHATOM);
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {  // 128 keys, 16 per MMA
+            const uint64_t ad = sdesc(vstage + kk * 2048, lbo, 1024, kLayoutSW128);
+            const uint64_t bd = sdesc(p_s + sb * C::P_BYTES + kk * 1024, C::P_BYTES, 512, kLayoutSW64);
+            umma_bf16_ss(tmem + 64, ad, bd, kIdescPV, (c == 0 && kk == 0) ? 0u : 1u);
+          }
+          umma_commit(&pc->vempty[vs]);
+          umma_commit(&pc->obar);
+        }
+      }
+      ++v_used;
+      ++pv_issued;
+      if (!(ok = all_ok(mine))) break;
+      mine = true;
     }
+    if (!ok) break;
 
     // ---- epilogue: O = O^T / l, LSE = (max + log2 l) ln 2
-    if (!warp_wait(&ctl->pv_done[slot], pv_waits & 1, &ctl->abort)) return;
-    ++pv_waits;
+    if (!(ok = all_ok(ensure_pv_done(pv_base + nch)))) break;
     tc_fence_after();
     uint32_t u[32];
     tmem_ld32(o_col, u);
     tmem_wait_ld();
     tc_fence_before();
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&ctl->o_free[slot]);
-    {
-      const float wsum = transpose_reduce(lpart, [](float x, float y) { return x + y; });
-      ctl->red[slot][warp][lane] = wsum;
-      named_bar(bar_id, 128);
-      if (warp == 0)
-        ctl->lsum[slot][lane] = (ctl->red[slot][0][lane] + ctl->red[slot][1][lane]) +
-                                (ctl->red[slot][2][lane] + ctl->red[slot][3][lane]);
-    }
+    const float wsum = transpose_reduce(lpart, [](float p, float s) { return p + s; });
+    pc->red[warp][lane] = wsum;
+    named_bar(bar_id, 128);
+    if (warp == 0)
+      pc->lsum[lane] = (pc->red[0][lane] + pc->red[1][lane]) + (pc->red[2][lane] + pc->red[3][lane]);
     named_bar(bar_id, 128);
     if (warp < D / 32) {
-      const int d = tid;  // O^T row = head-dim index
-      __nv_bfloat16* orow = a.O + row0 * D + d;
+      __nv_bfloat16* orow = a.O + row0 * D + tid;  // O^T row = head-dim index
 #pragma unroll
       for (int q = 0; q < 32; q += 4) {
-        const float4 l4 = *reinterpret_cast<const float4*>(&ctl->lsum[slot][q]);
+        const float4 l4 = *reinterpret_cast<const float4*>(&pc->lsum[q]);
         const float ls[4] = {l4.x, l4.y, l4.z, l4.w};
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const float inv = ls[i] > 0.f ? 1.f / ls[i] : 0.f;
-          orow[static_cast<long long>(q + i) * D] = __float2bfloat16_rn(__uint_as_float(u[q + i]) * inv);
+          orow[static_cast<long long>(q + i) * D] =
+              __float2bfloat16_rn(__uint_as_float(u[q + i]) * inv);
         }
       }
     }
     if (warp == 3) {
-      const float l = ctl->lsum[slot][lane];
+      const float l = pc->lsum[lane];
       a.LSE[row0 + lane] = l > 0.f ? (m_own + __log2f(l)) * 0.69314718055994531f : kNegInf;
     }
   }
+  // teardown: every MMA of this pipeline completes before the CTA ends
+  if (tid == 0) {
+    umma_commit(&pc->fbar);
+    wait_drain(&pc->fbar, 0);
+  }
+  __syncwarp();
 }
 
 template <int D>
-__global__ void __launch_bounds__(kThreads, 1)
-    fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-               const __grid_constant__ CUtensorMap tmV, const FwdArgs args) {
+__global__ void __launch_bounds__(Cfg<D>::THREADS, 1) fwd_kernel(const FwdArgs args) {
   using C = Cfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   Ctrl* ctl = reinterpret_cast<Ctrl*>(smem + C::OFF_CTRL);
   const int warp = threadIdx.x >> 5;
+  const int wgi = warp >> 2;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(&ctl->bm_full[s], 1);
-      mbar_init(&ctl->bm_empty[s], 6);  // softmax warps of the slot (4) + MMA + V producer
-      mbar_init(&ctl->q_full[s], 1);
-      mbar_init(&ctl->q_empty[s], 1);
-      mbar_init(&ctl->s_full[s], 1);
-      mbar_init(&ctl->s_free[s], 4);
-      mbar_init(&ctl->pv_done[s], 1);
-      mbar_init(&ctl->o_free[s], 4);
-      for (int b = 0; b < 4; ++b) {
-        mbar_init(&ctl->p_full[s][b], 4);
-        mbar_init(&ctl->p_empty[s][b], 1);
+    for (int w = 0; w < C::NWG; ++w) {
+      PipeCtrl* pc = &ctl->pipe[w];
+      for (int s = 0; s < 2; ++s) {
+        mbar_init(&pc->bm_full[s], 1);
+        mbar_init(&pc->bm_empty[s], 5);  // the 4 softmax warps and the V warp
+        mbar_init(&pc->sbar[s], 1);
       }
+      mbar_init(&pc->qfull, 32);
+      mbar_init(&pc->qempty, 1);
+      for (int s = 0; s < C::NKS; ++s) {
+        mbar_init(&pc->kfull[s], 32);
+        mbar_init(&pc->kempty[s], 1);
+      }
+      for (int s = 0; s < C::NVS; ++s) {
+        mbar_init(&pc->vfull[s], 32);
+        mbar_init(&pc->vempty[s], 1);
+      }
+      mbar_init(&pc->obar, 1);
+      mbar_init(&pc->fbar, 1);
     }
-    for (int s = 0; s < 4; ++s) {
-      mbar_init(&ctl->k_full[s], 1);
-      mbar_init(&ctl->k_empty[s], 1);
-      mbar_init(&ctl->v_full[s], 1);
-      mbar_init(&ctl->v_empty[s], 1);
-    }
-    mbar_init(&ctl->final_bar, 1);
     ctl->abort.v = 0;
     fence_mbar_init();
   }
-  if (warp < 8) {
-    // P^T buffers start at zero (a stale NaN pattern times a zero V row would
-    // still be NaN); for d = 64 the zero tile completes the O^T A operand.
-    uint4* p = reinterpret_cast<uint4*>(smem + C::OFF_P);
-    for (int i = threadIdx.x; i < 2 * C::NP * C::P_BYTES / 16; i += 256) p[i] = make_uint4(0u, 0u, 0u, 0u);
-    if constexpr (C::PAD_A) {
-      uint4* z = reinterpret_cast<uint4*>(smem + C::OFF_PAD);
-      for (int i = threadIdx.x; i < C::CHATOM / 16; i += 256) z[i] = make_uint4(0u, 0u, 0u, 0u);
-    }
-    fence_proxy_async_smem();
+  // P^T buffers start at zero (a stale NaN pattern times a zero V row would
+  // still be NaN); for d = 64 the zero tile completes the O^T A operand.
+  for (int w = 0; w < C::NWG; ++w) {
+    uint4* p = reinterpret_cast<uint4*>(smem + w * C::WG_BYTES + C::OFF_P);
+    for (int i = threadIdx.x; i < 2 * C::P_BYTES / 16; i += C::THREADS) p[i] = make_uint4(0u, 0u, 0u, 0u);
   }
-  if (warp == 10) {
-    tmem_alloc(&ctl->tmem_base, 512);
+  if constexpr (C::PAD_A) {
+    uint4* z = reinterpret_cast<uint4*>(smem + C::OFF_PAD);
+    for (int i = threadIdx.x; i < C::CHATOM / 16; i += C::THREADS) z[i] = make_uint4(0u, 0u, 0u, 0u);
+  }
+  fence_proxy_async_smem();
+  if (warp == 0) {
+    tmem_alloc(&ctl->tmem_base, C::TMEM_COLS);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -623,23 +654,27 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = ctl->tmem_base;
 
-  if (warp < 8) {
-    softmax_role<D>(args, smem, ctl, tmem, warp >> 2);
-    __syncwarp();
-  } else if (warp == 8) {
-    producer_qk<D>(&tmQ, &tmK, args, smem, ctl);
-  } else if (warp == 9) {
-    producer_v<D>(&tmV, args, smem, ctl);
+  if (wgi == C::COPY_WG) {
+    if constexpr (C::NWG > 1) setmaxnreg_dec<C::REGS_COPY>();
+    const int cw = warp & 3;  // copy warp: pipeline cw / 2, K (even) or V (odd)
+    const int pipe = cw >> 1;
+    if (pipe < C::NWG) {
+      uint8_t* base = smem + pipe * C::WG_BYTES;
+      if ((cw & 1) == 0)
+        copy_warp_qk<D>(args, base, &ctl->pipe[pipe], &ctl->abort, pipe);
+      else
+        copy_warp_v<D>(args, base, &ctl->pipe[pipe], &ctl->abort, pipe);
+    }
   } else {
-    if ((threadIdx.x & 31) == 0) mma_role<D>(args, smem, ctl, tmem);
-    __syncwarp();
+    if constexpr (C::NWG > 1) setmaxnreg_inc<C::REGS_SOFTMAX>();
+    softmax_wg<D>(args, smem, ctl, tmem, wgi);
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 10) {
+  if (warp == 0) {
     tc_fence_after();
-    tmem_dealloc(tmem, 512);
+    tmem_dealloc(tmem, C::TMEM_COLS);
   }
 }
 

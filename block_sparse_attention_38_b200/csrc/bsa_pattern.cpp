@@ -9,7 +9,7 @@
 #include <cstdint>
 #include <vector>
 
-#include "../../include/bsa.h"
+#include "bsa.h"
 
 namespace {
 
