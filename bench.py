@@ -46,11 +46,14 @@ METRIC = "block-sparse attn fwd useful TFLOP/s & ms/fwd (1 B200), % of roofline"
 DEFAULT_WORKLOAD = "loglinear_4k"
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-KERNEL_SOURCE = os.path.join(ROOT, "block_sparse_attention_38_b200", "csrc", "bsa_forward.cu")
+KERNEL_DIR = os.path.join(ROOT, "block_sparse_attention_38_b200", "csrc")
 
 # DRAM bytes (read + write) per launch from ncu captures of the kernel, keyed by
-# workload, valid only for the kernel source whose sha256 prefix is given.
-NCU_TRAFFIC = {}
+# workload, valid only for the kernel sources whose sha256 prefix is given
+# (profiles/ holds the capture summaries).
+NCU_TRAFFIC = {
+    "loglinear_4k": (25386240, "fa1f3368a6716f19"),
+}
 
 
 def useful_flops(w, nnz_all_heads: int) -> float:
@@ -62,8 +65,13 @@ def compulsory_bytes(w) -> float:
 
 
 def kernel_hash() -> str:
-    with open(KERNEL_SOURCE, "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+    """sha256 prefix over every kernel source file (sorted by name)."""
+    h = hashlib.sha256()
+    for name in sorted(os.listdir(KERNEL_DIR)):
+        if name.endswith((".cu", ".cuh")):
+            with open(os.path.join(KERNEL_DIR, name), "rb") as f:
+                h.update(name.encode() + b"\0" + f.read())
+    return h.hexdigest()[:16]
 
 
 def load_peaks():

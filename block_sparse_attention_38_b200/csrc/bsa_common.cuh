@@ -26,9 +26,6 @@ __device__ unsigned int g_status;
 struct FwdArgs {
   const int32_t* row_ptr;
   const int32_t* col_idx;
-  const __nv_bfloat16* Q;  // [B,H,N,d] (read with cp.async by the key-tile kernel)
-  const __nv_bfloat16* K;
-  const __nv_bfloat16* V;
   __nv_bfloat16* O;
   float* LSE;
   int H, N, M, G, W;      // G = tiles per (b, h); W = 32-bit words per block-row bitmap
@@ -104,13 +101,5 @@ struct BitIter {
   }
 };
 
-
-// Named barrier over `nthreads` threads (ids 1..15; id 0 is __syncthreads).
-// The warp is reconverged first and the non-aligned form is used, so a lane
-// that arrives after a divergent branch of its warp still counts correctly.
-__device__ __forceinline__ void named_bar(int id, int nthreads) {
-  __syncwarp();
-  asm volatile("barrier.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
-}
 
 }  // namespace bsa

@@ -1,12 +1,11 @@
 // bsa_forward.cu -- host side of the block-sparse attention forward: argument
-// validation, TMA descriptor encoding and the launch of one of two sm_100a
-// kernels (the key-tile kernel for 32-token blocks, the row-tile kernel for
-// 64- and 128-token blocks).  This file is the library's only CUDA
-// translation unit; the kernels live in the headers it includes.
+// validation, TMA descriptor encoding and the launch of the sm_100a row-tile
+// kernel (one instantiation per block size and head dimension).  This file is
+// the library's only CUDA translation unit; the kernel lives in the headers it
+// includes.
 #include <mutex>
 
 #include "bsa_common.cuh"
-#include "bsa_fwd_keys.cuh"
 #include "bsa_fwd_rows.cuh"
 
 namespace bsa {
@@ -85,8 +84,6 @@ int launch_rows(const void* Q, const void* K, const void* V, const int32_t* row_
   FwdArgs a;
   a.row_ptr = row_ptr;
   a.col_idx = col_idx;
-  a.K = static_cast<const __nv_bfloat16*>(K);
-  a.V = static_cast<const __nv_bfloat16*>(V);
   a.O = static_cast<__nv_bfloat16*>(O);
   a.LSE = LSE;
   a.H = H;
@@ -102,6 +99,11 @@ int launch_rows(const void* Q, const void* K, const void* V, const int32_t* row_
   const int smem_req = smem < 120 * 1024 ? 120 * 1024 : smem;
   static bool attr_set[64] = {};
   if (!attr_set[dev]) {
+    // The warpgroups trade registers (setmaxnreg); the kernel must have been
+    // built with the register count that the trade assumes.
+    cudaFuncAttributes fa;
+    if (cudaFuncGetAttributes(&fa, rows::fwd_kernel<BS, D>) != cudaSuccess) return BSA_ERR_CUDA;
+    if (fa.numRegs != rows::kRegsAtLaunch) return BSA_ERR_UNSUPPORTED;
     if (cudaFuncSetAttribute(rows::fwd_kernel<BS, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              smem_req) != cudaSuccess)
       return BSA_ERR_CUDA;
@@ -109,47 +111,6 @@ int launch_rows(const void* Q, const void* K, const void* V, const int32_t* row_
   }
   const long long grid = a.num_tiles < di.sms ? a.num_tiles : di.sms;
   rows::fwd_kernel<BS, D><<<static_cast<unsigned>(grid), rows::kThreads, smem_req, stream>>>(tq, tk, tv, a);
-  if (cudaGetLastError() != cudaSuccess) return BSA_ERR_CUDA;
-  return BSA_OK;
-}
-
-template <int D>
-int launch_keys(const void* Q, const void* K, const void* V, const int32_t* row_ptr,
-                const int32_t* col_idx, int B, int H, int N, float scale, int causal, void* O,
-                float* LSE, cudaStream_t stream) {
-  using C = keys::Cfg<D>;
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return BSA_ERR_CUDA;
-  DeviceInfo di;
-  if (!device_info(dev, &di)) return BSA_ERR_CUDA;
-  const long long BH = static_cast<long long>(B) * H;
-  FwdArgs a;
-  a.row_ptr = row_ptr;
-  a.col_idx = col_idx;
-  a.Q = static_cast<const __nv_bfloat16*>(Q);
-  a.K = static_cast<const __nv_bfloat16*>(K);
-  a.V = static_cast<const __nv_bfloat16*>(V);
-  a.O = static_cast<__nv_bfloat16*>(O);
-  a.LSE = LSE;
-  a.H = H;
-  a.N = N;
-  a.M = N / 32;
-  a.G = a.M;
-  a.W = (a.M + 31) / 32;
-  a.num_tiles = BH * a.M;
-  a.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
-  a.causal = causal;
-  const int smem = C::OFF_CTRL + static_cast<int>(sizeof(keys::Ctrl)) + 1024;
-  static bool attr_set[64] = {};
-  if (!attr_set[dev]) {
-    if (cudaFuncSetAttribute(keys::fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             smem) != cudaSuccess)
-      return BSA_ERR_CUDA;
-    attr_set[dev] = true;
-  }
-  const long long pipes = (a.num_tiles + C::NWG - 1) / C::NWG;
-  const long long grid = pipes < di.sms ? pipes : di.sms;
-  keys::fwd_kernel<D><<<static_cast<unsigned>(grid), C::THREADS, smem, stream>>>(a);
   if (cudaGetLastError() != cudaSuccess) return BSA_ERR_CUDA;
   return BSA_OK;
 }
@@ -176,8 +137,8 @@ extern "C" int bsa_forward(const void* Q, const void* K, const void* V, const in
   if (static_cast<long long>(H) * (N / block_size) + 1 > 2147483647LL) return BSA_ERR_UNSUPPORTED;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   switch (block_size * 1000 + d) {
-    case 32064: return launch_keys<64>(Q, K, V, row_ptr, col_idx, B, H, N, scale, causal, O, LSE, s);
-    case 32128: return launch_keys<128>(Q, K, V, row_ptr, col_idx, B, H, N, scale, causal, O, LSE, s);
+    case 32064: return launch_rows<32, 64>(Q, K, V, row_ptr, col_idx, B, H, N, scale, causal, O, LSE, s);
+    case 32128: return launch_rows<32, 128>(Q, K, V, row_ptr, col_idx, B, H, N, scale, causal, O, LSE, s);
     case 64064: return launch_rows<64, 64>(Q, K, V, row_ptr, col_idx, B, H, N, scale, causal, O, LSE, s);
     case 64128: return launch_rows<64, 128>(Q, K, V, row_ptr, col_idx, B, H, N, scale, causal, O, LSE, s);
     case 128064: return launch_rows<128, 64>(Q, K, V, row_ptr, col_idx, B, H, N, scale, causal, O, LSE, s);
