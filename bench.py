@@ -51,9 +51,7 @@ KERNEL_DIR = os.path.join(ROOT, "block_sparse_attention_38_b200", "csrc")
 # DRAM bytes (read + write) per launch from ncu captures of the kernel, keyed by
 # workload, valid only for the kernel sources whose sha256 prefix is given
 # (profiles/ holds the capture summaries).
-NCU_TRAFFIC = {
-    "loglinear_4k": (25386240, "fa1f3368a6716f19"),
-}
+NCU_TRAFFIC = {}
 
 
 def useful_flops(w, nnz_all_heads: int) -> float:

@@ -99,17 +99,13 @@ int launch_rows(const void* Q, const void* K, const void* V, const int32_t* row_
   const int smem_req = smem < 120 * 1024 ? 120 * 1024 : smem;
   static bool attr_set[64] = {};
   if (!attr_set[dev]) {
-    // The warpgroups trade registers (setmaxnreg); the kernel must have been
-    // built with the register count that the trade assumes.
-    cudaFuncAttributes fa;
-    if (cudaFuncGetAttributes(&fa, rows::fwd_kernel<BS, D>) != cudaSuccess) return BSA_ERR_CUDA;
-    if (fa.numRegs != rows::kRegsAtLaunch) return BSA_ERR_UNSUPPORTED;
     if (cudaFuncSetAttribute(rows::fwd_kernel<BS, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              smem_req) != cudaSuccess)
       return BSA_ERR_CUDA;
     attr_set[dev] = true;
   }
-  const long long grid = a.num_tiles < di.sms ? a.num_tiles : di.sms;
+  long long grid = a.num_tiles < di.sms ? a.num_tiles : di.sms;
+  if (grid > rows::kMaxGrid) grid = rows::kMaxGrid;
   rows::fwd_kernel<BS, D><<<static_cast<unsigned>(grid), rows::kThreads, smem_req, stream>>>(tq, tk, tv, a);
   if (cudaGetLastError() != cudaSuccess) return BSA_ERR_CUDA;
   return BSA_OK;

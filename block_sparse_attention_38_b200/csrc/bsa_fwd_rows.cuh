@@ -22,11 +22,11 @@
 // TMEM: slot s uses columns [256 s, 256 s + 128) for S (P aliases the first
 // 64) and [256 s + 128, 256 s + 128 + d) for the O accumulator.
 //
-// Work split: each CTA takes a contiguous range of tiles whose estimated cost
-// (longest row of the tile plus one step) sums to 1/grid of the total, so a
-// few very long rows (the global rows of the local+global pattern) do not
-// leave one SM finishing late; the CTA's two slots take tiles from that range
-// in turn through a shared-memory counter.
+// Work split (`schedule`): tiles whose estimated cost (longest row plus one
+// step) exceeds half of a CTA's share -- the global rows of the local+global
+// pattern -- are dealt out one per CTA first; the remaining tiles are cut into
+// contiguous ranges that fill each CTA's leftover share.  The CTA's two slots
+// take tiles from its list in turn through a shared-memory counter.
 #pragma once
 
 #include "bsa_common.cuh"
@@ -36,11 +36,6 @@ namespace rows {
 
 constexpr int kThreads = 384;
 constexpr int kSlots = 2;
-constexpr int kRegsSoftmax = 216;   // warpgroups 0 and 1
-constexpr int kRegsOther = 72;      // warpgroup 2 (producers, MMA issuers)
-constexpr int kRegsAtLaunch = 168;  // 65536 / 384 rounded down to a multiple of 8
-static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsOther <= kThreads * kRegsAtLaunch,
-              "register split exceeds the registers the CTA is launched with");
 
 template <int BS, int D>
 struct Cfg {
@@ -73,11 +68,26 @@ struct SlotCtrl {
   int n[2];           // union size (blocks) of each bitmap buffer
 };
 
+constexpr int kMaxGrid = 256;               // CTAs per launch (the host caps the grid)
+constexpr int kMaxHeavyGroups = 2 * kMaxGrid;
+
+// This CTA's work: up to two heavy tiles, then the light tiles of a
+// contiguous range (heavy tiles inside it belong to other CTAs and are skipped).
+struct Sched {
+  long long heavy[2];
+  long long light_begin, light_end;
+  long long thr;                    // a tile group whose cost exceeds thr is heavy (-1: none is)
+  long long scan[kThreads / 32];
+  int n_heavy;
+  int next_tile;                    // slots' shared cursor over heavy tiles, then light ones
+  int light_next;
+  int heavy_hg[kMaxHeavyGroups];    // heavy groups of one batch element, in order
+  int heavy_cost[kMaxHeavyGroups];
+};
+
 struct Ctrl {
   SlotCtrl slot[kSlots];
-  long long range_begin, range_end;
-  long long scan[kThreads / 32];
-  int next_tile;
+  Sched sched;
   uint32_t tmem_base;
   AbortFlag abort;
   uint32_t bitmap[kSlots][2][5 * kMaxBitmapWords];  // R block-row maps, then their union
@@ -100,55 +110,143 @@ __device__ __forceinline__ long long group_cost(const FwdArgs& a, long long hg) 
   return mx + R;
 }
 
-// All threads: the contiguous tile range [range_begin, range_end) of this CTA.
-// Tile T = (b*H + h)*G + g has prefix cost b*P + p(h*G + g), p the exclusive
-// prefix of group_cost over the H*G groups of one batch element and P their
-// sum; CTA c owns the tiles whose prefix lies in [c*total/grid, (c+1)*total/grid).
+// Block-wide exclusive scan of v (every thread calls it); *total = sum over the CTA.
+__device__ __forceinline__ long long block_scan(long long v, long long* total, long long* buf) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  long long incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const long long t = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += t;
+  }
+  __syncthreads();  // buf is free again
+  if (lane == 31) buf[warp] = incl;
+  __syncthreads();
+  long long base = 0, tot = 0;
+  for (int w = 0; w < kThreads / 32; ++w) {
+    const long long x = buf[w];
+    if (w < warp) base += x;
+    tot += x;
+  }
+  *total = tot;
+  return base + incl - v;
+}
+
+// All threads: this CTA's share of the tiles (the tile schedule).
+//
+// Tile T = (b*H + h)*G + g; its cost is group_cost of group hg = h*G + g (the
+// pattern is shared across b).  Every CTA computes the same plan:
+//  1. total = sum of all tile costs; a group is heavy when its cost exceeds
+//     thr = total / (2*grid), half of one CTA's share (so there are fewer than
+//     2*grid heavy tiles).
+//  2. Heavy tile k (in tile order) goes to CTA k mod grid.
+//  3. CTA c gets light capacity max(0, total/grid - its heavy cost); the light
+//     tiles are cut into contiguous ranges whose light-cost prefix falls in
+//     [L*Cap(c)/Cap, L*Cap(c+1)/Cap), Cap(c) the capacity of the CTAs before c.
+// The busiest CTA then carries at most max(its heavy tiles, share + one light
+// tile) instead of share + the largest tile.
 template <int BS>
-__device__ void compute_range(const FwdArgs& a, Ctrl* ctl) {
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+__device__ void schedule(const FwdArgs& a, Ctrl* ctl) {
+  Sched& sd = ctl->sched;
+  const int tid = threadIdx.x;
   const long long HG = static_cast<long long>(a.H) * a.G;
   const long long seg = (HG + kThreads - 1) / kThreads;
   const long long lo = min(HG, tid * seg), hi = min(HG, lo + seg);
+  const long long nb = a.num_tiles / HG;
+  const long long grid = gridDim.x;
+  const long long c = blockIdx.x;
+
   long long sum = 0;
   for (long long hg = lo; hg < hi; ++hg) sum += group_cost<BS>(a, hg);
-  long long incl = sum;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const long long v = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += v;
-  }
-  if (lane == 31) ctl->scan[warp] = incl;
-  __syncthreads();
-  long long base = 0, per_b = 0;
-  for (int w = 0; w < kThreads / 32; ++w) {
-    if (w < warp) base += ctl->scan[w];
-    per_b += ctl->scan[w];
-  }
-  const long long excl = base + incl - sum;
-  const long long nb = a.num_tiles / HG;
+  long long per_b;
+  block_scan(sum, &per_b, sd.scan);
   const long long total = per_b * nb;
-  const long long grid = gridDim.x;
+  const long long thr = total / (2 * grid);
+
+  long long n_hv = 0, lsum = 0;
+  for (long long hg = lo; hg < hi; ++hg) {
+    const long long cst = group_cost<BS>(a, hg);
+    if (cst > thr) ++n_hv; else lsum += cst;
+  }
+  long long Kg, Lper;
+  long long hexcl = block_scan(n_hv, &Kg, sd.scan);
+  const long long lexcl = block_scan(lsum, &Lper, sd.scan);
+  for (long long hg = lo; hg < hi && n_hv > 0; ++hg) {
+    const long long cst = group_cost<BS>(a, hg);
+    if (cst > thr) {
+      sd.heavy_hg[hexcl] = static_cast<int>(hg);
+      sd.heavy_cost[hexcl] = static_cast<int>(cst);
+      ++hexcl;
+    }
+  }
+  __syncthreads();
+  const long long Kh = Kg * nb;  // heavy tiles; Kh < 2*grid <= kMaxHeavyGroups
+  auto heavy_tile_cost = [&](long long k) -> long long { return k < Kh ? sd.heavy_cost[k % Kg] : 0; };
+
+  // Light capacity of the CTAs before this one, and of all of them.
+  const long long target = total / grid;
+  long long cap_before = 0, cap_all = 0, cap_mine = 0;
+  for (long long cc = tid; cc < grid; cc += kThreads) {
+    const long long hc = heavy_tile_cost(cc) + heavy_tile_cost(cc + grid);
+    const long long cap = hc < target ? target - hc : 0;
+    if (cc < c) cap_before += cap;
+    if (cc == c) cap_mine = cap;
+    cap_all += cap;
+  }
+  long long cap_b, cap_t, cap_m;
+  block_scan(cap_before, &cap_b, sd.scan);
+  block_scan(cap_all, &cap_t, sd.scan);
+  block_scan(cap_mine, &cap_m, sd.scan);
+
+  const long long L = Lper * nb;
   for (int e = 0; e < 2; ++e) {
-    const long long c = static_cast<long long>(blockIdx.x) + e;
-    const long long x = (total / grid) * c + ((total % grid) * c) / grid;
-    long long* out = e == 0 ? &ctl->range_begin : &ctl->range_end;
-    if (x >= total) {
+    const long long capx = cap_b + (e ? cap_m : 0);
+    long long x;
+    if (c + e == grid) x = L;
+    else if (cap_t > 0) x = static_cast<long long>(static_cast<__int128>(capx) * L / cap_t);
+    else x = static_cast<long long>(static_cast<__int128>(c + e) * L / grid);
+    long long* out = e == 0 ? &sd.light_begin : &sd.light_end;
+    if (x >= L) {
       if (tid == 0) *out = a.num_tiles;
       continue;
     }
-    const long long b = x / per_b, rem = x - b * per_b;
+    const long long b = x / Lper, rem = x - b * Lper;
     if (rem == 0) {
       if (tid == 0) *out = b * HG;
       continue;
     }
-    if (excl < rem && rem <= excl + sum) {
-      long long run = excl, hg = lo;
-      while (run < rem) run += group_cost<BS>(a, hg++);
+    if (lexcl < rem && rem <= lexcl + lsum) {
+      long long run = lexcl, hg = lo;
+      while (run < rem) {
+        const long long cst = group_cost<BS>(a, hg++);
+        run += cst > thr ? 0 : cst;
+      }
       *out = b * HG + hg;
     }
   }
+  if (tid == 0) {
+    int nh = 0;
+    for (long long k = c; k < Kh && nh < 2; k += grid)
+      sd.heavy[nh++] = (k / Kg) * HG + sd.heavy_hg[k % Kg];
+    sd.n_heavy = nh;
+    sd.thr = Kh > 0 ? thr : -1;  // -1: no heavy tile exists, nothing to skip
+    sd.next_tile = 0;
+    sd.light_next = 0;
+  }
   __syncthreads();
+}
+
+// Next tile for a slot of this CTA (producer lane 0), -1 when none is left.
+template <int BS>
+__device__ __forceinline__ long long next_tile(const FwdArgs& a, Sched& sd) {
+  const int i = atomicAdd(&sd.next_tile, 1);
+  if (i < sd.n_heavy) return sd.heavy[i];
+  const long long HG = static_cast<long long>(a.H) * a.G;
+  for (;;) {
+    const long long t = sd.light_begin + atomicAdd(&sd.light_next, 1);
+    if (t >= sd.light_end) return -1;
+    if (sd.thr < 0 || group_cost<BS>(a, t % HG) <= sd.thr) return t;
+  }
 }
 
 // ------------------------------------------------------------ producer warp
@@ -175,8 +273,7 @@ __device__ void load_role(int s, const CUtensorMap* tmQ, const CUtensorMap* tmK,
     if (lane == 0) {
       w_ok = wait_bounded(&sc.bm_empty[buf], ((t >> 1) & 1) ^ 1, &ctl->abort);
       if (w_ok) {
-        tile = ctl->range_begin + atomicAdd(&ctl->next_tile, 1);
-        if (tile >= ctl->range_end) tile = -1;
+        tile = next_tile<BS>(a, ctl->sched);
       }
     }
     if (!__shfl_sync(0xffffffffu, w_ok, 0)) { ok = false; break; }
@@ -391,40 +488,47 @@ __device__ void softmax_role(int s, const FwdArgs& a, Ctrl* ctl, uint32_t tmem) 
     float l = 0.f;           // running sum of 2^(s - m_used)
     BitIter it(bm + C::R * a.W, a.W);
     for (int j = 0; j < steps; ++j) {
-      int jb[C::BPS];
-      bool val[C::BPS];
-      bool any = false;
+      // Blocks of this step: vmask bit b = this row holds block b of the step,
+      // dmask bit b = block b is this row's diagonal block under causal masking.
+      uint32_t vmask = 0, dmask = 0;
 #pragma unroll
       for (int b = 0; b < C::BPS; ++b) {
-        jb[b] = it.next();
-        val[b] = row_ok && jb[b] >= 0 && ((mine[jb[b] >> 5] >> (jb[b] & 31)) & 1u);
-        any = any || val[b];
+        const int jb = it.next();
+        if (row_ok && jb >= 0 && ((mine[jb >> 5] >> (jb & 31)) & 1u)) vmask |= 1u << b;
+        if (a.causal && jb == r_sub) dmask |= 1u << b;
       }
       if (!warp_wait(&sc.s_full, s_seen & 1, &ctl->abort)) return;
       ++s_seen;
       tc_fence_after();
-      uint32_t x[128];
-      if (any) {
-        // All four column groups are loaded even when some blocks are masked:
-        // a conditional tcgen05.ld leaves its registers undefined on one path,
-        // which makes the compiler spill the whole score row.
-#pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_ld32(t_s + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&x[c * 32]));
-        tmem_wait_ld();
-#pragma unroll
-        for (int c = 0; c < 4; ++c) reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&x[c * 32]));
-
+      // The 128 scores are taken in four groups of 32 columns (group g covers
+      // keys 32g..32g+31, block g*32/BS); a group is read from TMEM once for
+      // the maximum and once for the exponentials, and its 16 packed P
+      // columns are written over S columns already consumed.
+      if (vmask != 0) {  // uniform over the warp
         float mx = kNegInf;
+#pragma unroll 1
+        for (int gp = 0; gp < 2; ++gp) {
+          const int b0 = (2 * gp) * 32 / BS, b1 = (2 * gp + 1) * 32 / BS;
+          const bool ok0 = (vmask >> b0) & 1u, ok1 = (vmask >> b1) & 1u;
+          if (!ok0 && !ok1) continue;
+          uint32_t u[64];
+          tmem_ld32(t_s + gp * 64, *reinterpret_cast<uint32_t(*)[32]>(&u[0]));
+          tmem_ld32(t_s + gp * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&u[32]));
+          tmem_wait_ld();
+          reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&u[0]));
+          reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&u[32]));
 #pragma unroll
-        for (int b = 0; b < C::BPS; ++b) {
-          if (!val[b]) continue;
-          const bool diag = a.causal && jb[b] == r_sub;
+          for (int h = 0; h < 2; ++h) {
+            const int b = h ? b1 : b0;
+            if (!(h ? ok1 : ok0)) continue;
+            const bool diag = (dmask >> b) & 1u;
+            const int c0 = ((2 * gp + h) * 32) % BS;
 #pragma unroll
-          for (int c = 0; c < BS; ++c) {
-            float v = __uint_as_float(x[b * BS + c]) * sl2;
-            if (diag && c > qq) v = kNegInf;  // key after the query (diagonal block only)
-            x[b * BS + c] = __float_as_uint(v);
-            mx = fmaxf(mx, v);
+            for (int i = 0; i < 32; ++i) {
+              float v = __uint_as_float(u[h * 32 + i]) * sl2;
+              if (diag && c0 + i > qq) v = kNegInf;
+              mx = fmaxf(mx, v);
+            }
           }
         }
         float factor = 1.f;
@@ -439,7 +543,7 @@ __device__ void softmax_role(int s, const FwdArgs& a, Ctrl* ctl, uint32_t tmem) 
         }
         // The commit behind s_full also covers the previous PV: O is final here.
         if (__any_sync(0xffffffffu, need_rescale)) {
-#pragma unroll
+#pragma unroll 1
           for (int c = 0; c < D / 32; ++c) {
             uint32_t u[32];
             tmem_ld32(t_o + c * 32, u);
@@ -452,28 +556,50 @@ __device__ void softmax_role(int s, const FwdArgs& a, Ctrl* ctl, uint32_t tmem) 
         }
         const float mu = m_used == kNegInf ? 0.f : m_used;
         float rs = 0.f;
-#pragma unroll
-        for (int b = 0; b < C::BPS; ++b) {
-#pragma unroll
-          for (int c = 0; c < BS; ++c) {
-            float p = 0.f;
-            if (val[b]) {
-              p = ex2_approx(__uint_as_float(x[b * BS + c]) - mu);
-              rs += p;
-            }
-            x[b * BS + c] = __float_as_uint(p);
+#pragma unroll 1
+        for (int gp = 0; gp < 2; ++gp) {
+          const int b0 = (2 * gp) * 32 / BS, b1 = (2 * gp + 1) * 32 / BS;
+          const bool ok0 = (vmask >> b0) & 1u, ok1 = (vmask >> b1) & 1u;
+          uint32_t pk[32];
+          uint32_t u[64];
+          if (ok0 || ok1) {
+            tmem_ld32(t_s + gp * 64, *reinterpret_cast<uint32_t(*)[32]>(&u[0]));
+            tmem_ld32(t_s + gp * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&u[32]));
+            tmem_wait_ld();
+            reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&u[0]));
+            reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&u[32]));
           }
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int b = h ? b1 : b0;
+            if (h ? ok1 : ok0) {
+              const bool diag = (dmask >> b) & 1u;
+              const int c0 = ((2 * gp + h) * 32) % BS;
+#pragma unroll
+              for (int i = 0; i < 32; i += 2) {
+                float v0 = __uint_as_float(u[h * 32 + i]) * sl2, v1 = __uint_as_float(u[h * 32 + i + 1]) * sl2;
+                if (diag && c0 + i > qq) v0 = kNegInf;
+                if (diag && c0 + i + 1 > qq) v1 = kNegInf;
+                const float p0 = ex2_approx(v0 - mu), p1 = ex2_approx(v1 - mu);
+                rs += p0;
+                rs += p1;
+                pk[h * 16 + i / 2] = pack_bf16x2(p0, p1);
+              }
+            } else {
+#pragma unroll
+              for (int i = 0; i < 16; ++i) pk[h * 16 + i] = 0u;
+            }
+          }
+          tmem_st32(t_s + gp * 32, pk);
         }
         l = l * factor + rs;
-#pragma unroll
-        for (int i = 0; i < 64; ++i)
-          x[i] = pack_bf16x2(__uint_as_float(x[2 * i]), __uint_as_float(x[2 * i + 1]));
       } else {
+        uint32_t z[32];
 #pragma unroll
-        for (int i = 0; i < 64; ++i) x[i] = 0u;
+        for (int i = 0; i < 32; ++i) z[i] = 0u;
+        tmem_st32(t_s, z);
+        tmem_st32(t_s + 32, z);
       }
-      tmem_st32(t_s, *reinterpret_cast<uint32_t(*)[32]>(&x[0]));
-      tmem_st32(t_s + 32, *reinterpret_cast<uint32_t(*)[32]>(&x[32]));
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
@@ -487,29 +613,31 @@ __device__ void softmax_role(int s, const FwdArgs& a, Ctrl* ctl, uint32_t tmem) 
       if (!warp_wait(&sc.o_full, o_seen & 1, &ctl->abort)) return;
       ++o_seen;
       tc_fence_after();
-      uint32_t o[D];
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+      uint4* dst = reinterpret_cast<uint4*>(orow);
+#pragma unroll 1
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t u[32];
+        tmem_ld32(t_o + c * 32, u);
+        tmem_wait_ld();
+        reg_fence32(u);
+        if (row_ok) {
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) tmem_ld32(t_o + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&o[c * 32]));
-      tmem_wait_ld();
-#pragma unroll
-      for (int c = 0; c < D / 32; ++c) reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&o[c * 32]));
+          for (int q = 0; q < 4; ++q) {
+            uint4 v;
+            v.x = pack_bf16x2(__uint_as_float(u[q * 8 + 0]) * inv, __uint_as_float(u[q * 8 + 1]) * inv);
+            v.y = pack_bf16x2(__uint_as_float(u[q * 8 + 2]) * inv, __uint_as_float(u[q * 8 + 3]) * inv);
+            v.z = pack_bf16x2(__uint_as_float(u[q * 8 + 4]) * inv, __uint_as_float(u[q * 8 + 5]) * inv);
+            v.w = pack_bf16x2(__uint_as_float(u[q * 8 + 6]) * inv, __uint_as_float(u[q * 8 + 7]) * inv);
+            dst[c * 4 + q] = v;
+          }
+        }
+      }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sc.o_empty);
-      if (row_ok) {
-        const float inv = l > 0.f ? 1.f / l : 0.f;
-        uint4* dst = reinterpret_cast<uint4*>(orow);
-#pragma unroll
-        for (int c = 0; c < D / 8; ++c) {
-          uint4 v;
-          v.x = pack_bf16x2(__uint_as_float(o[c * 8 + 0]) * inv, __uint_as_float(o[c * 8 + 1]) * inv);
-          v.y = pack_bf16x2(__uint_as_float(o[c * 8 + 2]) * inv, __uint_as_float(o[c * 8 + 3]) * inv);
-          v.z = pack_bf16x2(__uint_as_float(o[c * 8 + 4]) * inv, __uint_as_float(o[c * 8 + 5]) * inv);
-          v.w = pack_bf16x2(__uint_as_float(o[c * 8 + 6]) * inv, __uint_as_float(o[c * 8 + 7]) * inv);
-          dst[c] = v;
-        }
+      if (row_ok)
         a.LSE[bh * a.N + qtok] = l > 0.f ? (m_used + __log2f(l)) * 0.69314718055994531f : kNegInf;
-      }
     } else if (row_ok) {
       uint4* dst = reinterpret_cast<uint4*>(orow);
 #pragma unroll
@@ -551,7 +679,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&sc.o_empty, 4);
       mbar_init(&sc.final_bar, 1);
     }
-    ctl->next_tile = 0;
     ctl->abort.v = 0;
     fence_mbar_init();
   }
@@ -559,18 +686,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(&ctl->tmem_base, C::TMEM_COLS);
     tmem_relinquish();
   }
-  compute_range<BS>(args, ctl);
+  schedule<BS>(args, ctl);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = ctl->tmem_base;
 
   if (warp < 8) {
-    setmaxnreg_inc<kRegsSoftmax>();
     softmax_role<BS, D>(warp >> 2, args, ctl, tmem);
     __syncwarp();
   } else {
-    setmaxnreg_dec<kRegsOther>();
     if (warp < 10) {
       load_role<BS, D>(warp - 8, &tmQ, &tmK, &tmV, args, smem, ctl);
     } else {
