@@ -29,7 +29,8 @@ MUTANTS = {
     "v_row_index": ("const uint16_t *vrow = V + (head * N + keys[i]) * (int64_t)d;",
                     "const uint16_t *vrow = V + (head * N + q) * (int64_t)d;"),
     "block_to_token_index": ("int64_t k = (int64_t)j * bs + t;", "int64_t k = (int64_t)j + t;"),
-    "block_row_of_query": ("const int64_t r = q / bs;", "const int64_t r = (q + 1) / bs;"),
+    # an off-by-one that stays inside [0, M): (q - 1) / bs truncates to 0 at q = 0
+    "block_row_of_query": ("const int64_t r = q / bs;", "const int64_t r = (q - 1) / bs;"),
     "no_normalisation": ("const double w = score[i] / l;", "const double w = score[i];"),
     "duplicates_counted": ("if (seen[j]) continue;", ";"),
     "lse_without_max": ("*lse = m + log(l);", "*lse = log(l);"),
@@ -47,7 +48,15 @@ def _compile(tmp_path, name, text):
 
 
 def _pins_pass(lib):
-    """True when every pin holds for this library."""
+    """True when every pin holds for this library (a mutant that reports an
+    error instead of a result fails them too)."""
+    try:
+        return _pins_hold(lib)
+    except ValueError:
+        return False
+
+
+def _pins_hold(lib):
     rng = np.random.default_rng(1234)
     # brute force, plain and causal, with duplicated column entries
     for causal in (False, True):
