@@ -5,8 +5,7 @@
 // of 128 keys (128 / block_size blocks gathered into one shared-memory stage):
 //
 //   S = Q K_step^T            tcgen05.mma, M=128 queries, N=128 keys, K=d
-//   P = 2^(S*scale*log2e - m) one thread per query row, fp32, written back to
-//                             TMEM as bf16 over the first half of S
+//   P = 2^(S*scale*log2e - m) fp32 in registers, written back to TMEM as bf16
 //   O += P V_step             tcgen05.mma with A = P read from TMEM, N=d
 //
 // A block row that does not hold a block of the step gets P = 0 there and its
@@ -14,19 +13,30 @@
 // Sparse Attention with Log-Linear Complexity", section 3.3); the exponentials
 // of such blocks are not evaluated (membership is uniform over a warp).
 //
-// One persistent CTA per SM runs two independent tile slots so that the
-// tensor core works on one slot while the other slot's softmax runs.  Roles:
-//   warps 0-3   softmax / epilogue of slot 0    warps 4-7  same, slot 1
-//   warp 8 + s  bitmap builder + TMA producer of slot s
-//   warp 10 + s tcgen05.mma issuer of slot s (warp 10 also owns the TMEM)
-// TMEM: slot s uses columns [256 s, 256 s + 128) for S (P aliases the first
-// 64) and [256 s + 128, 256 s + 128 + d) for the O accumulator.
+// One persistent CTA per SM.  S and O are double-buffered in TMEM, so the MMA
+// issuer runs one step ahead of the softmax: while the softmax turns S(j)
+// into P(j), the tensor core computes S(j+1); then O += P(j) V(j) and S(j+2).
+// The next tile's first steps overlap the previous tile's epilogue the same
+// way.  Roles (384 threads):
+//   warps 0-3   softmax, columns 0-63 of every step (keys 0..63), and the
+//               epilogue of O columns [0, d/2)
+//   warps 4-7   the same for columns 64-127 and O columns [d/2, d)
+//   warp 8      tile schedule, per-tile block bitmaps, TMA loads of Q, K, V
+//   warp 9      tcgen05.mma issuer (and owner of the 512 TMEM columns)
+// The two softmax warpgroups cover the same 128 rows (TMEM lane quadrant
+// warp % 4); per step they exchange the row maximum of their halves through
+// shared memory (an mbarrier with bounded waits, not a hardware barrier, so
+// that a warpgroup giving up cannot leave the other waiting), so both use the
+// same running maximum; their partial sums are added at the end of the tile.
+//
+// TMEM columns: S(j) in [128 (j&1), +128); P(j) over the columns already
+// read: keys 0..63 at [128 (j&1), +32), keys 64..127 at [128 (j&1) + 64, +32);
+// O of tile t in [256 + d (t&1), +d).
 //
 // Work split (`schedule`): tiles whose estimated cost (longest row plus one
 // step) exceeds half of a CTA's share -- the global rows of the local+global
 // pattern -- are dealt out one per CTA first; the remaining tiles are cut into
-// contiguous ranges that fill each CTA's leftover share.  The CTA's two slots
-// take tiles from its list in turn through a shared-memory counter.
+// contiguous ranges that fill each CTA's leftover share.
 #pragma once
 
 #include "bsa_common.cuh"
@@ -35,7 +45,6 @@ namespace bsa {
 namespace rows {
 
 constexpr int kThreads = 384;
-constexpr int kSlots = 2;
 
 template <int BS, int D>
 struct Cfg {
@@ -46,51 +55,54 @@ struct Cfg {
   static constexpr int KATOMS = D / 64;          // 128-byte column atoms of a D-wide row
   static constexpr int Q_BYTES = TM * D * 2;
   static constexpr int CH_BYTES = NK * D * 2;    // one K or V stage
-  static constexpr int NKS = D == 64 ? 2 : 1;    // K stages per slot
-  static constexpr int NVS = D == 64 ? 2 : 1;    // V stages per slot
-  static constexpr int SLOT_KV = (NKS + NVS) * CH_BYTES;
-  static constexpr int OFF_Q = 0;                // + slot * Q_BYTES
-  static constexpr int OFF_KV = kSlots * Q_BYTES;  // + slot * SLOT_KV: K stages, then V stages
-  static constexpr int OFF_CTRL = OFF_KV + kSlots * SLOT_KV;
+  static constexpr int NKS = D == 64 ? 3 : 2;    // K stages
+  static constexpr int NVS = D == 64 ? 3 : 2;    // V stages
+  static constexpr int OFF_Q = 0;                // two Q buffers
+  static constexpr int OFF_K = 2 * Q_BYTES;
+  static constexpr int OFF_V = OFF_K + NKS * CH_BYTES;
+  static constexpr int OFF_CTRL = OFF_V + NVS * CH_BYTES;
   static constexpr uint32_t TMEM_COLS = 512;
-  static constexpr uint32_t TMEM_SLOT = 256;
-  static constexpr uint32_t TMEM_O = 128;
+  static constexpr uint32_t TMEM_O = 256;
   static_assert((Q_BYTES % 1024) == 0 && (CH_BYTES % 1024) == 0, "1024-byte aligned stages");
-};
-
-struct SlotCtrl {
-  uint64_t bm_full[2], bm_empty[2];
-  uint64_t q_full, q_empty;
-  uint64_t k_full[2], k_empty[2], v_full[2], v_empty[2];
-  uint64_t s_full, p_full, o_full, o_empty;
-  uint64_t final_bar;
-  long long tile[2];  // tile index of each bitmap buffer, -1 = no more work
-  int n[2];           // union size (blocks) of each bitmap buffer
+  static_assert(TMEM_O + 2 * D <= TMEM_COLS, "TMEM layout");
+  static_assert(TM == NK, "Q and K tiles share one slice-offset formula");
 };
 
 constexpr int kMaxGrid = 256;               // CTAs per launch (the host caps the grid)
 constexpr int kMaxHeavyGroups = 2 * kMaxGrid;
 
-// This CTA's work: up to two heavy tiles, then the light tiles of a
-// contiguous range (heavy tiles inside it belong to other CTAs and are skipped).
+// This CTA's work (see `schedule`).
 struct Sched {
-  long long heavy[2];
-  long long light_begin, light_end;
-  long long thr;                    // a tile group whose cost exceeds thr is heavy (-1: none is)
+  long long heavy[2];               // this CTA's heavy tiles
+  long long n_light;                // light tiles in all
+  long long kh;                     // heavy tiles in all
   long long scan[kThreads / 32];
   int n_heavy;
-  int next_tile;                    // slots' shared cursor over heavy tiles, then light ones
-  int light_next;
+  int skip;                         // rounds of light tiles a CTA holding a heavy tile sits out
+  int kg;                           // heavy groups per batch element
+  // producer-side cursor
+  int next_heavy;
+  long long round;                  // next round of light tiles
+  long long hp;                     // heavy tiles known to lie before the current light tile
   int heavy_hg[kMaxHeavyGroups];    // heavy groups of one batch element, in order
   int heavy_cost[kMaxHeavyGroups];
 };
 
 struct Ctrl {
-  SlotCtrl slot[kSlots];
+  uint64_t bm_full[2], bm_empty[2];
+  uint64_t q_full[2], q_empty[2];
+  uint64_t k_full[3], k_empty[3], v_full[3], v_empty[3];
+  uint64_t s_full[2], p_full[2], pv_done[2];
+  uint64_t o_full[2], o_empty[2];
+  uint64_t xbar[2];   // exchanges between the two softmax warpgroups
+  uint64_t final_bar;
+  long long tile[2];  // tile index of each bitmap buffer, -1 = no more work
+  int n[2];           // union size (blocks) of each bitmap buffer
   Sched sched;
   uint32_t tmem_base;
   AbortFlag abort;
-  uint32_t bitmap[kSlots][2][5 * kMaxBitmapWords];  // R block-row maps, then their union
+  float red[2][2][128];      // [exchange parity][half][row]: partial row max or sum
+  uint32_t bitmap[2][5 * kMaxBitmapWords];  // R block-row maps, then their union
 };
 
 // Estimated cost of tile group (h, g) in blocks: the longest of its rows, plus
@@ -136,15 +148,14 @@ __device__ __forceinline__ long long block_scan(long long v, long long* total, l
 //
 // Tile T = (b*H + h)*G + g; its cost is group_cost of group hg = h*G + g (the
 // pattern is shared across b).  Every CTA computes the same plan:
-//  1. total = sum of all tile costs; a group is heavy when its cost exceeds
-//     thr = total / (2*grid), half of one CTA's share (so there are fewer than
-//     2*grid heavy tiles).
-//  2. Heavy tile k (in tile order) goes to CTA k mod grid.
-//  3. CTA c gets light capacity max(0, total/grid - its heavy cost); the light
-//     tiles are cut into contiguous ranges whose light-cost prefix falls in
-//     [L*Cap(c)/Cap, L*Cap(c+1)/Cap), Cap(c) the capacity of the CTAs before c.
-// The busiest CTA then carries at most max(its heavy tiles, share + one light
-// tile) instead of share + the largest tile.
+//  1. total = sum of the tile costs; a tile is heavy when its cost exceeds
+//     thr = total / (2*grid), half of one CTA's share, so there are fewer than
+//     2*grid heavy tiles.  Heavy tile k (in tile order) goes to CTA k mod grid.
+//  2. The other ("light") tiles, in tile order, are dealt out in rounds of
+//     one tile per CTA, so that the CTAs work on neighbouring tiles at any
+//     time and share the K/V blocks those tiles read in L2.
+//  3. When there are at most `grid` heavy tiles, the CTAs holding one sit out
+//     the first `skip` rounds, skip = average heavy cost / average light cost.
 template <int BS>
 __device__ void schedule(const FwdArgs& a, Ctrl* ctl) {
   Sched& sd = ctl->sched;
@@ -163,14 +174,17 @@ __device__ void schedule(const FwdArgs& a, Ctrl* ctl) {
   const long long total = per_b * nb;
   const long long thr = total / (2 * grid);
 
-  long long n_hv = 0, lsum = 0;
+  long long n_hv = 0, hsum = 0;
   for (long long hg = lo; hg < hi; ++hg) {
     const long long cst = group_cost<BS>(a, hg);
-    if (cst > thr) ++n_hv; else lsum += cst;
+    if (cst > thr) {
+      ++n_hv;
+      hsum += cst;
+    }
   }
-  long long Kg, Lper;
+  long long Kg, Hper;
   long long hexcl = block_scan(n_hv, &Kg, sd.scan);
-  const long long lexcl = block_scan(lsum, &Lper, sd.scan);
+  block_scan(hsum, &Hper, sd.scan);
   for (long long hg = lo; hg < hi && n_hv > 0; ++hg) {
     const long long cst = group_cost<BS>(a, hg);
     if (cst > thr) {
@@ -179,86 +193,76 @@ __device__ void schedule(const FwdArgs& a, Ctrl* ctl) {
       ++hexcl;
     }
   }
-  __syncthreads();
-  const long long Kh = Kg * nb;  // heavy tiles; Kh < 2*grid <= kMaxHeavyGroups
-  auto heavy_tile_cost = [&](long long k) -> long long { return k < Kh ? sd.heavy_cost[k % Kg] : 0; };
-
-  // Light capacity of the CTAs before this one, and of all of them.
-  const long long target = total / grid;
-  long long cap_before = 0, cap_all = 0, cap_mine = 0;
-  for (long long cc = tid; cc < grid; cc += kThreads) {
-    const long long hc = heavy_tile_cost(cc) + heavy_tile_cost(cc + grid);
-    const long long cap = hc < target ? target - hc : 0;
-    if (cc < c) cap_before += cap;
-    if (cc == c) cap_mine = cap;
-    cap_all += cap;
-  }
-  long long cap_b, cap_t, cap_m;
-  block_scan(cap_before, &cap_b, sd.scan);
-  block_scan(cap_all, &cap_t, sd.scan);
-  block_scan(cap_mine, &cap_m, sd.scan);
-
-  const long long L = Lper * nb;
-  for (int e = 0; e < 2; ++e) {
-    const long long capx = cap_b + (e ? cap_m : 0);
-    long long x;
-    if (c + e == grid) x = L;
-    else if (cap_t > 0) x = static_cast<long long>(static_cast<__int128>(capx) * L / cap_t);
-    else x = static_cast<long long>(static_cast<__int128>(c + e) * L / grid);
-    long long* out = e == 0 ? &sd.light_begin : &sd.light_end;
-    if (x >= L) {
-      if (tid == 0) *out = a.num_tiles;
-      continue;
-    }
-    const long long b = x / Lper, rem = x - b * Lper;
-    if (rem == 0) {
-      if (tid == 0) *out = b * HG;
-      continue;
-    }
-    if (lexcl < rem && rem <= lexcl + lsum) {
-      long long run = lexcl, hg = lo;
-      while (run < rem) {
-        const long long cst = group_cost<BS>(a, hg++);
-        run += cst > thr ? 0 : cst;
-      }
-      *out = b * HG + hg;
-    }
-  }
   if (tid == 0) {
+    const long long Kh = Kg * nb;  // < 2*grid <= kMaxHeavyGroups
+    const long long n_light = a.num_tiles - Kh;
     int nh = 0;
     for (long long k = c; k < Kh && nh < 2; k += grid)
       sd.heavy[nh++] = (k / Kg) * HG + sd.heavy_hg[k % Kg];
+    long long skip = 0;
+    if (Kh > 0 && Kh <= grid && n_light > 0) {
+      const double heavy_avg = static_cast<double>(Hper * nb) / Kh;
+      const double light_avg = static_cast<double>(total - Hper * nb) / n_light;
+      skip = static_cast<long long>(heavy_avg / light_avg + 0.5);
+      const long long most = n_light / (grid - Kh > 0 ? grid - Kh : 1);
+      if (skip > most) skip = most;
+      if (grid - Kh <= 0) skip = 0;
+    }
     sd.n_heavy = nh;
-    sd.thr = Kh > 0 ? thr : -1;  // -1: no heavy tile exists, nothing to skip
-    sd.next_tile = 0;
-    sd.light_next = 0;
+    sd.kh = Kh;
+    sd.kg = static_cast<int>(Kg);
+    sd.n_light = n_light;
+    sd.skip = static_cast<int>(skip);
+    sd.next_heavy = 0;
+    sd.round = 0;
+    sd.hp = 0;
   }
   __syncthreads();
 }
 
-// Next tile for a slot of this CTA (producer lane 0), -1 when none is left.
+// Next tile of this CTA (producer lane 0), -1 when none is left: its heavy
+// tiles first, then its light tiles in increasing order.
 template <int BS>
 __device__ __forceinline__ long long next_tile(const FwdArgs& a, Sched& sd) {
-  const int i = atomicAdd(&sd.next_tile, 1);
-  if (i < sd.n_heavy) return sd.heavy[i];
-  const long long HG = static_cast<long long>(a.H) * a.G;
-  for (;;) {
-    const long long t = sd.light_begin + atomicAdd(&sd.light_next, 1);
-    if (t >= sd.light_end) return -1;
-    if (sd.thr < 0 || group_cost<BS>(a, t % HG) <= sd.thr) return t;
+  if (sd.next_heavy < sd.n_heavy) return sd.heavy[sd.next_heavy++];
+  const long long grid = gridDim.x, c = blockIdx.x;
+  const long long Kh = sd.kh;
+  const bool skipping = sd.skip > 0;             // at most grid heavy tiles, CTAs 0..Kh-1 hold one
+  const long long others = grid - Kh;            // CTAs without a heavy tile
+  const long long k = sd.round++;
+  long long i;                                   // index among the light tiles
+  if (!skipping) {
+    i = k * grid + c;
+  } else if (k < sd.skip) {
+    if (c < Kh) {                                // sits out the first rounds
+      sd.round = sd.skip + 1;
+      i = static_cast<long long>(sd.skip) * others + c;
+    } else {
+      i = k * others + (c - Kh);
+    }
+  } else {
+    i = static_cast<long long>(sd.skip) * others + (k - sd.skip) * grid + c;
   }
+  if (i >= sd.n_light) return -1;
+  // Light tile i is tile i + (heavy tiles before it); the heavy tiles are in
+  // increasing tile order and i only grows, so the count is kept across calls.
+  const long long HG = static_cast<long long>(a.H) * a.G;
+  long long t = i + sd.hp;
+  while (sd.hp < Kh && (sd.hp / sd.kg) * HG + sd.heavy_hg[sd.hp % sd.kg] <= t) {
+    ++sd.hp;
+    t = i + sd.hp;
+  }
+  return t;
 }
 
 // ------------------------------------------------------------ producer warp
+// Builds each tile's bitmaps (all lanes) and issues the TMA loads (lane 0) in
+// the order the MMA issuer consumes them: Q, then K(j), V(j) for every step.
 template <int BS, int D>
-__device__ void load_role(int s, const CUtensorMap* tmQ, const CUtensorMap* tmK,
-                          const CUtensorMap* tmV, const FwdArgs& a, uint8_t* smem, Ctrl* ctl) {
+__device__ void load_role(const CUtensorMap* tmQ, const CUtensorMap* tmK, const CUtensorMap* tmV,
+                          const FwdArgs& a, uint8_t* smem, Ctrl* ctl) {
   using C = Cfg<BS, D>;
-  SlotCtrl& sc = ctl->slot[s];
   const int lane = threadIdx.x & 31;
-  uint8_t* q_s = smem + C::OFF_Q + s * C::Q_BYTES;
-  uint8_t* k_s = smem + C::OFF_KV + s * C::SLOT_KV;
-  uint8_t* v_s = k_s + C::NKS * C::CH_BYTES;
   uint32_t q_loads = 0, k_loads = 0, v_loads = 0;
   bool ok = true;
   if (lane == 0) {
@@ -271,15 +275,13 @@ __device__ void load_role(int s, const CUtensorMap* tmQ, const CUtensorMap* tmK,
     int w_ok = 1;
     long long tile = -1;
     if (lane == 0) {
-      w_ok = wait_bounded(&sc.bm_empty[buf], ((t >> 1) & 1) ^ 1, &ctl->abort);
-      if (w_ok) {
-        tile = next_tile<BS>(a, ctl->sched);
-      }
+      w_ok = wait_bounded(&ctl->bm_empty[buf], ((t >> 1) & 1) ^ 1, &ctl->abort);
+      if (w_ok) tile = next_tile<BS>(a, ctl->sched);
     }
     if (!__shfl_sync(0xffffffffu, w_ok, 0)) { ok = false; break; }
     tile = __shfl_sync(0xffffffffu, tile, 0);
 
-    uint32_t* bm = ctl->bitmap[s][buf];
+    uint32_t* bm = ctl->bitmap[buf];
     const int W = a.W;
     long long bh = 0;
     int n = 0;
@@ -314,23 +316,24 @@ __device__ void load_role(int s, const CUtensorMap* tmQ, const CUtensorMap* tmK,
       n = union_count(bm + C::R * W, W);
     }
     if (lane == 0) {
-      sc.tile[buf] = tile;
-      sc.n[buf] = n;
+      ctl->tile[buf] = tile;
+      ctl->n[buf] = n;
     }
     __syncwarp();
-    if (lane == 0) mbar_arrive(&sc.bm_full[buf]);
+    if (lane == 0) mbar_arrive(&ctl->bm_full[buf]);
     if (tile < 0) break;
     if (n == 0) continue;
 
     if (lane == 0) {
       const int g = static_cast<int>(tile - bh * a.G);
-      ok = wait_bounded(&sc.q_empty, (q_loads & 1) ^ 1, &ctl->abort);
+      const uint32_t qb = q_loads & 1;
+      ok = wait_bounded(&ctl->q_empty[qb], ((q_loads >> 1) & 1) ^ 1, &ctl->abort);
       if (ok) {
-        mbar_arrive_expect_tx(&sc.q_full, C::Q_BYTES);
+        mbar_arrive_expect_tx(&ctl->q_full[qb], C::Q_BYTES);
 #pragma unroll
         for (int ka = 0; ka < C::KATOMS; ++ka)
-          tma_load_3d(q_s + ka * (C::TM * 128), tmQ, &sc.q_full, ka * 64, g * C::TM,
-                      static_cast<int>(bh));
+          tma_load_3d(smem + C::OFF_Q + qb * C::Q_BYTES + ka * (C::TM * 128), tmQ, &ctl->q_full[qb],
+                      ka * 64, g * C::TM, static_cast<int>(bh));
         ++q_loads;
       }
       BitIter it(bm + C::R * W, W);
@@ -343,26 +346,26 @@ __device__ void load_role(int s, const CUtensorMap* tmQ, const CUtensorMap* tmK,
           row0[b] = jb >= 0 ? jb * BS : a.N;
         }
         const uint32_t ks = k_loads % C::NKS;
-        ok = wait_bounded(&sc.k_empty[ks], ((k_loads / C::NKS) & 1) ^ 1, &ctl->abort);
+        ok = wait_bounded(&ctl->k_empty[ks], ((k_loads / C::NKS) & 1) ^ 1, &ctl->abort);
         if (!ok) break;
-        mbar_arrive_expect_tx(&sc.k_full[ks], C::CH_BYTES);
+        mbar_arrive_expect_tx(&ctl->k_full[ks], C::CH_BYTES);
 #pragma unroll
         for (int b = 0; b < C::BPS; ++b)
 #pragma unroll
           for (int ka = 0; ka < C::KATOMS; ++ka)
-            tma_load_3d(k_s + ks * C::CH_BYTES + ka * (C::NK * 128) + b * (BS * 128), tmK,
-                        &sc.k_full[ks], ka * 64, row0[b], static_cast<int>(bh));
+            tma_load_3d(smem + C::OFF_K + ks * C::CH_BYTES + ka * (C::NK * 128) + b * (BS * 128), tmK,
+                        &ctl->k_full[ks], ka * 64, row0[b], static_cast<int>(bh));
         ++k_loads;
         const uint32_t vs = v_loads % C::NVS;
-        ok = wait_bounded(&sc.v_empty[vs], ((v_loads / C::NVS) & 1) ^ 1, &ctl->abort);
+        ok = wait_bounded(&ctl->v_empty[vs], ((v_loads / C::NVS) & 1) ^ 1, &ctl->abort);
         if (!ok) break;
-        mbar_arrive_expect_tx(&sc.v_full[vs], C::CH_BYTES);
+        mbar_arrive_expect_tx(&ctl->v_full[vs], C::CH_BYTES);
 #pragma unroll
         for (int b = 0; b < C::BPS; ++b)
 #pragma unroll
           for (int ka = 0; ka < C::KATOMS; ++ka)
-            tma_load_3d(v_s + vs * C::CH_BYTES + ka * (C::NK * 128) + b * (BS * 128), tmV,
-                        &sc.v_full[vs], ka * 64, row0[b], static_cast<int>(bh));
+            tma_load_3d(smem + C::OFF_V + vs * C::CH_BYTES + ka * (C::NK * 128) + b * (BS * 128), tmV,
+                        &ctl->v_full[vs], ka * 64, row0[b], static_cast<int>(bh));
         ++v_loads;
       }
     }
@@ -370,282 +373,315 @@ __device__ void load_role(int s, const CUtensorMap* tmQ, const CUtensorMap* tmK,
   }
   // On an early exit, let every copy already issued land before the CTA ends.
   if (!ok && lane == 0) {
-    if (q_loads > 0) wait_drain(&sc.q_full, (q_loads - 1) & 1);
+    for (uint32_t b = 0; b < 2; ++b)
+      if (q_loads > b) {
+        const uint32_t last = b + 2 * ((q_loads - 1 - b) / 2);
+        wait_drain(&ctl->q_full[b], (last >> 1) & 1);
+      }
     for (uint32_t st = 0; st < C::NKS; ++st)
       if (k_loads > st) {
         const uint32_t last = st + C::NKS * ((k_loads - 1 - st) / C::NKS);
-        wait_drain(&sc.k_full[st], (last / C::NKS) & 1);
+        wait_drain(&ctl->k_full[st], (last / C::NKS) & 1);
       }
     for (uint32_t st = 0; st < C::NVS; ++st)
       if (v_loads > st) {
         const uint32_t last = st + C::NVS * ((v_loads - 1 - st) / C::NVS);
-        wait_drain(&sc.v_full[st], (last / C::NVS) & 1);
+        wait_drain(&ctl->v_full[st], (last / C::NVS) & 1);
       }
   }
   __syncwarp();
 }
 
 // ---------------------------------------------------------------- MMA issuer
-// Per step: S = Q K^T, then (once the softmax has written P) O += P V.  The
-// QK of the next step is issued right after the PV of this one: MMAs of one
-// thread run in issue order, so it overwrites S/P only after the PV read P,
-// and the commit that reports it also reports that PV.
+// Issue order within a tile of n steps: S(0), S(1), then for j = 0..n-1:
+// O += P(j) V(j) and S(j+2).  MMAs of one thread run in issue order, so S(j+2)
+// overwrites S(j)/P(j) only after the PV of step j has read P(j), and each
+// commit also reports every MMA issued before it.
 template <int BS, int D>
-__device__ void mma_role(int s, const FwdArgs& a, uint8_t* smem, Ctrl* ctl, uint32_t tmem) {
+__device__ void mma_role(const FwdArgs& a, uint8_t* smem, Ctrl* ctl, uint32_t tmem) {
   using C = Cfg<BS, D>;
-  SlotCtrl& sc = ctl->slot[s];
   constexpr uint32_t kIdescQK = idesc_bf16_f32(128, C::NK, false, false);  // Q, K K-major
   constexpr uint32_t kIdescPV = idesc_bf16_f32(128, D, false, true);       // V MN-major
-  const uint32_t q_base = smem_u32(smem + C::OFF_Q + s * C::Q_BYTES);
-  const uint32_t k_base = smem_u32(smem + C::OFF_KV + s * C::SLOT_KV);
-  const uint32_t v_base = k_base + C::NKS * C::CH_BYTES;
-  const uint32_t t_s = tmem + s * C::TMEM_SLOT;
-  const uint32_t t_o = t_s + C::TMEM_O;
-  uint32_t k_cons = 0, v_cons = 0, q_uses = 0, p_seen = 0, o_tiles = 0;
+  const uint32_t q_base = smem_u32(smem + C::OFF_Q);
+  const uint32_t k_base = smem_u32(smem + C::OFF_K);
+  const uint32_t v_base = smem_u32(smem + C::OFF_V);
+  uint32_t k_cons = 0, v_cons = 0, q_uses = 0, o_tiles = 0, gstep = 0;
   bool ok = true;
   for (int t = 0; ok; ++t) {
     const int buf = t & 1;
-    if (!wait_bounded(&sc.bm_full[buf], (t >> 1) & 1, &ctl->abort)) break;
-    const long long tile = sc.tile[buf];
-    const int n = sc.n[buf];
-    mbar_arrive(&sc.bm_empty[buf]);
+    if (!wait_bounded(&ctl->bm_full[buf], (t >> 1) & 1, &ctl->abort)) break;
+    const long long tile = ctl->tile[buf];
+    const int n = ctl->n[buf];
+    mbar_arrive(&ctl->bm_empty[buf]);
     if (tile < 0) break;
     if (n == 0) continue;
     const int steps = (n + C::BPS - 1) / C::BPS;
-    if (!wait_bounded(&sc.q_full, q_uses & 1, &ctl->abort)) break;
+    const uint32_t qb = q_uses & 1;
+    if (!wait_bounded(&ctl->q_full[qb], (q_uses >> 1) & 1, &ctl->abort)) break;
     ++q_uses;
-    for (int j = 0; j < steps; ++j) {
+    const uint32_t ob = o_tiles & 1;
+    const uint32_t t_o = tmem + C::TMEM_O + ob * D;
+    const uint32_t q_tile = q_base + qb * C::Q_BYTES;
+
+    auto issue_qk = [&](int j) -> bool {
+      const uint32_t sb = (gstep + j) & 1;
       const uint32_t ks = k_cons % C::NKS;
-      if (!wait_bounded(&sc.k_full[ks], (k_cons / C::NKS) & 1, &ctl->abort)) { ok = false; break; }
+      if (!wait_bounded(&ctl->k_full[ks], (k_cons / C::NKS) & 1, &ctl->abort)) return false;
       tc_fence_after();
+      // Descriptors of consecutive K=16 slices differ only in the start
+      // address field (address >> 4), so they are a base plus a constant.
+      const uint64_t ad0 = sdesc_sw128(q_tile, 16, 1024);
+      const uint64_t bd0 = sdesc_sw128(k_base + ks * C::CH_BYTES, 16, 1024);
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk) {
-        const uint64_t ad = sdesc_sw128(q_base + (kk >> 2) * (C::TM * 128) + (kk & 3) * 32, 16, 1024);
-        const uint64_t bd = sdesc_sw128(
-            k_base + ks * C::CH_BYTES + (kk >> 2) * (C::NK * 128) + (kk & 3) * 32, 16, 1024);
-        umma_bf16_ss(t_s, ad, bd, kIdescQK, kk > 0 ? 1u : 0u);
+        const uint32_t off = ((kk >> 2) * (C::TM * 128) + (kk & 3) * 32) >> 4;  // TM == NK
+        umma_bf16_ss(tmem + sb * 128, ad0 + off, bd0 + off, kIdescQK, kk > 0 ? 1u : 0u);
       }
-      umma_commit(&sc.k_empty[ks]);
-      umma_commit(&sc.s_full);
-      if (j == steps - 1) umma_commit(&sc.q_empty);
+      umma_commit(&ctl->k_empty[ks]);
+      umma_commit(&ctl->s_full[sb]);
+      if (j == steps - 1) umma_commit(&ctl->q_empty[qb]);
       ++k_cons;
-
-      if (!wait_bounded(&sc.p_full, p_seen & 1, &ctl->abort)) { ok = false; break; }
-      ++p_seen;
+      return true;
+    };
+    auto issue_pv = [&](int j) -> bool {
+      const uint32_t gs = gstep + j, sb = gs & 1;
+      if (!wait_bounded(&ctl->p_full[sb], (gs >> 1) & 1, &ctl->abort)) return false;
       const uint32_t vs = v_cons % C::NVS;
-      if (!wait_bounded(&sc.v_full[vs], (v_cons / C::NVS) & 1, &ctl->abort)) { ok = false; break; }
-      if (j == 0 && o_tiles > 0 &&
-          !wait_bounded(&sc.o_empty, (o_tiles - 1) & 1, &ctl->abort)) { ok = false; break; }
+      if (!wait_bounded(&ctl->v_full[vs], (v_cons / C::NVS) & 1, &ctl->abort)) return false;
+      if (j == 0 && o_tiles >= 2 &&
+          !wait_bounded(&ctl->o_empty[ob], ((o_tiles - 2) >> 1) & 1, &ctl->abort))
+        return false;
       tc_fence_after();
+      const uint64_t bd0 = sdesc_sw128(v_base + vs * C::CH_BYTES, C::NK * 128, 1024);
+      const uint32_t a0 = tmem + sb * 128;
 #pragma unroll
       for (int kk = 0; kk < C::NK / 16; ++kk) {
-        const uint64_t bd =
-            sdesc_sw128(v_base + vs * C::CH_BYTES + kk * (16 * 128), C::NK * 128, 1024);
-        umma_bf16_ts(t_o, t_s + kk * 8, bd, kIdescPV, (j > 0 || kk > 0) ? 1u : 0u);
+        // P of keys 16kk..16kk+15: columns 8kk (keys < 64) or 64 + 8(kk-4) (keys >= 64).
+        const uint32_t a_col = kk < 4 ? kk * 8 : 64 + (kk - 4) * 8;
+        umma_bf16_ts(t_o, a0 + a_col, bd0 + ((kk * 16 * 128) >> 4), kIdescPV,
+                     (j > 0 || kk > 0) ? 1u : 0u);
       }
-      umma_commit(&sc.v_empty[vs]);
+      umma_commit(&ctl->v_empty[vs]);
+      umma_commit(&ctl->pv_done[sb]);
+      if (j == steps - 1) umma_commit(&ctl->o_full[ob]);
       ++v_cons;
-      if (j == steps - 1) umma_commit(&sc.o_full);
-    }
+      return true;
+    };
+
+    ok = issue_qk(0) && (steps < 2 || issue_qk(1));
+    for (int j = 0; ok && j < steps; ++j) ok = issue_pv(j) && (j + 2 >= steps || issue_qk(j + 2));
+    gstep += steps;
     ++o_tiles;
   }
   // Every MMA issued must complete before the TMEM is released.
-  umma_commit(&sc.final_bar);
-  wait_drain(&sc.final_bar, 0);
+  umma_commit(&ctl->final_bar);
+  wait_drain(&ctl->final_bar, 0);
 }
 
 // ------------------------------------------------------------ softmax warps
+// Warpgroup `half` handles keys 64*half .. 64*half+63 of every step (two
+// groups of 32 TMEM columns) for all 128 rows, and O columns
+// [half*d/2, (half+1)*d/2) in the epilogue.
 template <int BS, int D>
-__device__ void softmax_role(int s, const FwdArgs& a, Ctrl* ctl, uint32_t tmem) {
+__device__ void softmax_role(int half, const FwdArgs& a, Ctrl* ctl, uint32_t tmem) {
   using C = Cfg<BS, D>;
-  SlotCtrl& sc = ctl->slot[s];
-  const int row = threadIdx.x - s * 128;  // query row of the tile
-  const int warp = row >> 5;
-  const int lane = row & 31;
-  const int sub = row / BS;               // block row of the tile this thread belongs to
-  const int qq = row % BS;                // position inside that block row
-  const uint32_t t_s = tmem + s * C::TMEM_SLOT + (static_cast<uint32_t>(warp * 32) << 16);
-  const uint32_t t_o = t_s + C::TMEM_O;
+  constexpr int HD = D / 2;                    // O columns of this warpgroup
+  const int wq = (threadIdx.x >> 5) & 3;       // TMEM lane quadrant
+  const int lane = threadIdx.x & 31;
+  const int row = wq * 32 + lane;              // query row of the tile
+  const int sub = row / BS;                    // block row of the tile this thread belongs to
+  const int qq = row % BS;                     // position inside that block row
+  const uint32_t t_lane = static_cast<uint32_t>(wq * 32) << 16;
   const float sl2 = a.scale_log2;
   constexpr float kNegInf = -INFINITY;
-  uint32_t s_seen = 0, o_seen = 0;
+  uint32_t gstep = 0, o_tiles = 0, n_ex = 0;
+  // Both warpgroups have written their values for exchange number n_ex:
+  // every warp arrives on xbar[n_ex & 1] (eight warps in all) and waits for
+  // the phase (bounded).  Values live in buffer n_ex & 1, so the next write
+  // to a buffer comes after the other warpgroup has passed the exchange that
+  // read it.
+  auto exchange = [&]() -> bool {
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&ctl->xbar[n_ex & 1]);
+    const bool ok = warp_wait(&ctl->xbar[n_ex & 1], (n_ex >> 1) & 1, &ctl->abort);
+    return ok;
+  };
 
   for (int t = 0;; ++t) {
     const int buf = t & 1;
-    if (!warp_wait(&sc.bm_full[buf], (t >> 1) & 1, &ctl->abort)) return;
-    const long long tile = sc.tile[buf];
-    const int n = sc.n[buf];
+    if (!warp_wait(&ctl->bm_full[buf], (t >> 1) & 1, &ctl->abort)) return;
+    const long long tile = ctl->tile[buf];
+    const int n = ctl->n[buf];
     if (tile < 0) return;
-    const uint32_t* bm = ctl->bitmap[s][buf];
+    const uint32_t* bm = ctl->bitmap[buf];
     const uint32_t* mine = bm + sub * a.W;
     const long long bh = tile / a.G;
     const int g = static_cast<int>(tile - bh * a.G);
     const int r_sub = g * C::R + sub;
     const bool row_ok = r_sub < a.M;
     const int steps = (n + C::BPS - 1) / C::BPS;
+    const long long qtok = static_cast<long long>(g) * C::TM + row;
+    uint4* orow = reinterpret_cast<uint4*>(a.O + (bh * a.N + qtok) * D + half * HD);
 
-    float m_used = kNegInf;  // running max, log2 units of the scaled score
-    float l = 0.f;           // running sum of 2^(s - m_used)
+    if (n == 0) {
+      if (row_ok) {
+#pragma unroll
+        for (int c = 0; c < HD / 8; ++c) orow[c] = make_uint4(0u, 0u, 0u, 0u);
+        if (half == 0) a.LSE[bh * a.N + qtok] = kNegInf;
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ctl->bm_empty[buf]);
+      continue;
+    }
+
+    float m_used = kNegInf;  // running max, log2 units of the scaled score (same in both halves)
+    float l = 0.f;           // this half's running sum of 2^(s - m_used)
     BitIter it(bm + C::R * a.W, a.W);
     for (int j = 0; j < steps; ++j) {
-      // Blocks of this step: vmask bit b = this row holds block b of the step,
-      // dmask bit b = block b is this row's diagonal block under causal masking.
+      const uint32_t gs = gstep + j, sb = gs & 1;
+      // This half's two 32-column groups: vmask bit i = the row holds the
+      // block of group i, dmask bit i = that block is its causal diagonal.
       uint32_t vmask = 0, dmask = 0;
 #pragma unroll
       for (int b = 0; b < C::BPS; ++b) {
         const int jb = it.next();
-        if (row_ok && jb >= 0 && ((mine[jb >> 5] >> (jb & 31)) & 1u)) vmask |= 1u << b;
-        if (a.causal && jb == r_sub) dmask |= 1u << b;
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+          if ((2 * half + i) * 32 / BS != b) continue;
+          if (row_ok && jb >= 0 && ((mine[jb >> 5] >> (jb & 31)) & 1u)) vmask |= 1u << i;
+          if (a.causal && jb == r_sub) dmask |= 1u << i;
+        }
       }
-      if (!warp_wait(&sc.s_full, s_seen & 1, &ctl->abort)) return;
-      ++s_seen;
+      if (!warp_wait(&ctl->s_full[sb], (gs >> 1) & 1, &ctl->abort)) return;
       tc_fence_after();
-      // The 128 scores are taken in four groups of 32 columns (group g covers
-      // keys 32g..32g+31, block g*32/BS); a group is read from TMEM once for
-      // the maximum and once for the exponentials, and its 16 packed P
-      // columns are written over S columns already consumed.
+      const uint32_t t_s = tmem + t_lane + sb * 128 + half * 64;
+      uint32_t u[64];
+      float pmax = kNegInf;
       if (vmask != 0) {  // uniform over the warp
-        float mx = kNegInf;
+        tmem_ld32(t_s, *reinterpret_cast<uint32_t(*)[32]>(&u[0]));
+        tmem_ld32(t_s + 32, *reinterpret_cast<uint32_t(*)[32]>(&u[32]));
+        tmem_wait_ld();
+        reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&u[0]));
+        reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&u[32]));
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+          if (!((vmask >> i) & 1u)) continue;
+          const bool diag = (dmask >> i) & 1u;
+          const int c0 = ((2 * half + i) * 32) % BS;  // first column of the group inside its block
+#pragma unroll
+          for (int c = 0; c < 32; ++c) {
+            float v = __uint_as_float(u[i * 32 + c]) * sl2;
+            if (diag && c0 + c > qq) v = kNegInf;  // key after the query (diagonal block only)
+            u[i * 32 + c] = __float_as_uint(v);
+            pmax = fmaxf(pmax, v);
+          }
+        }
+      }
+      // Row maximum over both halves.
+      ctl->red[n_ex & 1][half][row] = pmax;
+      if (!exchange()) return;
+      const float mx = fmaxf(pmax, ctl->red[n_ex & 1][half ^ 1][row]);
+      ++n_ex;
+
+      // Lazy rescale: the running maximum moves only when the step's maximum
+      // exceeds it by more than the threshold (P stays <= 2^8 otherwise).
+      float factor = 1.f;
+      bool need_rescale = false;
+      if (mx > m_used + kRescaleThreshold) {
+        if (m_used != kNegInf) {
+          need_rescale = true;
+          factor = ex2_approx(m_used - mx);
+        }
+        m_used = mx;
+      }
+      if (__any_sync(0xffffffffu, need_rescale)) {
+        // O must hold every PV up to the previous step.
+        const uint32_t pg = gs - 1;
+        if (!warp_wait(&ctl->pv_done[pg & 1], (pg >> 1) & 1, &ctl->abort)) return;
+        tc_fence_after();
+        const uint32_t t_o = tmem + t_lane + C::TMEM_O + (o_tiles & 1) * D + half * HD;
 #pragma unroll 1
-        for (int gp = 0; gp < 2; ++gp) {
-          const int b0 = (2 * gp) * 32 / BS, b1 = (2 * gp + 1) * 32 / BS;
-          const bool ok0 = (vmask >> b0) & 1u, ok1 = (vmask >> b1) & 1u;
-          if (!ok0 && !ok1) continue;
-          uint32_t u[64];
-          tmem_ld32(t_s + gp * 64, *reinterpret_cast<uint32_t(*)[32]>(&u[0]));
-          tmem_ld32(t_s + gp * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&u[32]));
+        for (int c = 0; c < HD / 32; ++c) {
+          uint32_t w[32];
+          tmem_ld32(t_o + c * 32, w);
           tmem_wait_ld();
-          reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&u[0]));
-          reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&u[32]));
+          reg_fence32(w);
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const int b = h ? b1 : b0;
-            if (!(h ? ok1 : ok0)) continue;
-            const bool diag = (dmask >> b) & 1u;
-            const int c0 = ((2 * gp + h) * 32) % BS;
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              float v = __uint_as_float(u[h * 32 + i]) * sl2;
-              if (diag && c0 + i > qq) v = kNegInf;
-              mx = fmaxf(mx, v);
-            }
-          }
+          for (int i = 0; i < 32; ++i) w[i] = __float_as_uint(__uint_as_float(w[i]) * factor);
+          tmem_st32(t_o + c * 32, w);
         }
-        float factor = 1.f;
-        bool need_rescale = false;
-        const float m_new = fmaxf(m_used, mx);
-        if (m_new > m_used + kRescaleThreshold) {
-          if (l > 0.f) {
-            need_rescale = true;
-            factor = ex2_approx(m_used - m_new);
-          }
-          m_used = m_new;
-        }
-        // The commit behind s_full also covers the previous PV: O is final here.
-        if (__any_sync(0xffffffffu, need_rescale)) {
-#pragma unroll 1
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t u[32];
-            tmem_ld32(t_o + c * 32, u);
-            tmem_wait_ld();
-            reg_fence32(u);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) u[i] = __float_as_uint(__uint_as_float(u[i]) * factor);
-            tmem_st32(t_o + c * 32, u);
-          }
-        }
+      }
+      l *= factor;
+
+      uint32_t pk[32];
+      if (vmask != 0) {
         const float mu = m_used == kNegInf ? 0.f : m_used;
         float rs = 0.f;
-#pragma unroll 1
-        for (int gp = 0; gp < 2; ++gp) {
-          const int b0 = (2 * gp) * 32 / BS, b1 = (2 * gp + 1) * 32 / BS;
-          const bool ok0 = (vmask >> b0) & 1u, ok1 = (vmask >> b1) & 1u;
-          uint32_t pk[32];
-          uint32_t u[64];
-          if (ok0 || ok1) {
-            tmem_ld32(t_s + gp * 64, *reinterpret_cast<uint32_t(*)[32]>(&u[0]));
-            tmem_ld32(t_s + gp * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&u[32]));
-            tmem_wait_ld();
-            reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&u[0]));
-            reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&u[32]));
-          }
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const int b = h ? b1 : b0;
-            if (h ? ok1 : ok0) {
-              const bool diag = (dmask >> b) & 1u;
-              const int c0 = ((2 * gp + h) * 32) % BS;
+        for (int i = 0; i < 2; ++i) {
+          const bool on = (vmask >> i) & 1u;
 #pragma unroll
-              for (int i = 0; i < 32; i += 2) {
-                float v0 = __uint_as_float(u[h * 32 + i]) * sl2, v1 = __uint_as_float(u[h * 32 + i + 1]) * sl2;
-                if (diag && c0 + i > qq) v0 = kNegInf;
-                if (diag && c0 + i + 1 > qq) v1 = kNegInf;
-                const float p0 = ex2_approx(v0 - mu), p1 = ex2_approx(v1 - mu);
-                rs += p0;
-                rs += p1;
-                pk[h * 16 + i / 2] = pack_bf16x2(p0, p1);
-              }
-            } else {
-#pragma unroll
-              for (int i = 0; i < 16; ++i) pk[h * 16 + i] = 0u;
+          for (int c = 0; c < 32; c += 2) {
+            float p0 = 0.f, p1 = 0.f;
+            if (on) {
+              p0 = ex2_approx(__uint_as_float(u[i * 32 + c]) - mu);
+              p1 = ex2_approx(__uint_as_float(u[i * 32 + c + 1]) - mu);
+              rs += p0;
+              rs += p1;
             }
+            pk[i * 16 + c / 2] = pack_bf16x2(p0, p1);
           }
-          tmem_st32(t_s + gp * 32, pk);
         }
-        l = l * factor + rs;
+        l += rs;
       } else {
-        uint32_t z[32];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) z[i] = 0u;
-        tmem_st32(t_s, z);
-        tmem_st32(t_s + 32, z);
+        for (int i = 0; i < 32; ++i) pk[i] = 0u;
       }
+      tmem_st32(tmem + t_lane + sb * 128 + half * 64, pk);  // P columns of this half
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&sc.p_full);
+      if (lane == 0) mbar_arrive(&ctl->p_full[sb]);
     }
 
-    // Epilogue: O / l in bf16 and LSE = (m + log2 l) ln 2.
-    const long long qtok = static_cast<long long>(g) * C::TM + row;
-    __nv_bfloat16* orow = a.O + (bh * a.N + qtok) * D;
-    if (n > 0) {
-      if (!warp_wait(&sc.o_full, o_seen & 1, &ctl->abort)) return;
-      ++o_seen;
-      tc_fence_after();
-      const float inv = l > 0.f ? 1.f / l : 0.f;
-      uint4* dst = reinterpret_cast<uint4*>(orow);
+    // Epilogue: O / l in bf16 (this half's columns) and LSE = (m + log2 l) ln 2.
+    ctl->red[n_ex & 1][half][row] = l;
+    if (!exchange()) return;
+    const float lt = l + ctl->red[n_ex & 1][half ^ 1][row];
+    ++n_ex;
+    const uint32_t ob = o_tiles & 1;
+    if (!warp_wait(&ctl->o_full[ob], (o_tiles >> 1) & 1, &ctl->abort)) return;
+    tc_fence_after();
+    const float inv = lt > 0.f ? 1.f / lt : 0.f;
+    const uint32_t t_o = tmem + t_lane + C::TMEM_O + ob * D + half * HD;
 #pragma unroll 1
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t u[32];
-        tmem_ld32(t_o + c * 32, u);
-        tmem_wait_ld();
-        reg_fence32(u);
-        if (row_ok) {
+    for (int c = 0; c < HD / 32; ++c) {
+      uint32_t w[32];
+      tmem_ld32(t_o + c * 32, w);
+      tmem_wait_ld();
+      reg_fence32(w);
+      if (row_ok) {
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            uint4 v;
-            v.x = pack_bf16x2(__uint_as_float(u[q * 8 + 0]) * inv, __uint_as_float(u[q * 8 + 1]) * inv);
-            v.y = pack_bf16x2(__uint_as_float(u[q * 8 + 2]) * inv, __uint_as_float(u[q * 8 + 3]) * inv);
-            v.z = pack_bf16x2(__uint_as_float(u[q * 8 + 4]) * inv, __uint_as_float(u[q * 8 + 5]) * inv);
-            v.w = pack_bf16x2(__uint_as_float(u[q * 8 + 6]) * inv, __uint_as_float(u[q * 8 + 7]) * inv);
-            dst[c * 4 + q] = v;
-          }
+        for (int q = 0; q < 4; ++q) {
+          uint4 v;
+          v.x = pack_bf16x2(__uint_as_float(w[q * 8 + 0]) * inv, __uint_as_float(w[q * 8 + 1]) * inv);
+          v.y = pack_bf16x2(__uint_as_float(w[q * 8 + 2]) * inv, __uint_as_float(w[q * 8 + 3]) * inv);
+          v.z = pack_bf16x2(__uint_as_float(w[q * 8 + 4]) * inv, __uint_as_float(w[q * 8 + 5]) * inv);
+          v.w = pack_bf16x2(__uint_as_float(w[q * 8 + 6]) * inv, __uint_as_float(w[q * 8 + 7]) * inv);
+          orow[c * 4 + q] = v;
         }
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&sc.o_empty);
-      if (row_ok)
-        a.LSE[bh * a.N + qtok] = l > 0.f ? (m_used + __log2f(l)) * 0.69314718055994531f : kNegInf;
-    } else if (row_ok) {
-      uint4* dst = reinterpret_cast<uint4*>(orow);
-#pragma unroll
-      for (int c = 0; c < D / 8; ++c) dst[c] = make_uint4(0u, 0u, 0u, 0u);
-      a.LSE[bh * a.N + qtok] = kNegInf;
     }
+    tc_fence_before();
     __syncwarp();
-    if (lane == 0) mbar_arrive(&sc.bm_empty[buf]);
+    if (lane == 0) {
+      mbar_arrive(&ctl->o_empty[ob]);
+      mbar_arrive(&ctl->bm_empty[buf]);
+    }
+    if (half == 0 && row_ok)
+      a.LSE[bh * a.N + qtok] = lt > 0.f ? (m_used + __log2f(lt)) * 0.69314718055994531f : kNegInf;
+    gstep += steps;
+    ++o_tiles;
   }
 }
 
@@ -661,28 +697,29 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kSlots; ++s) {
-      SlotCtrl& sc = ctl->slot[s];
-      for (int b = 0; b < 2; ++b) {
-        mbar_init(&sc.bm_full[b], 1);
-        mbar_init(&sc.bm_empty[b], 5);  // four softmax warps + the MMA issuer
-        mbar_init(&sc.k_full[b], 1);
-        mbar_init(&sc.k_empty[b], 1);
-        mbar_init(&sc.v_full[b], 1);
-        mbar_init(&sc.v_empty[b], 1);
-      }
-      mbar_init(&sc.q_full, 1);
-      mbar_init(&sc.q_empty, 1);
-      mbar_init(&sc.s_full, 1);
-      mbar_init(&sc.p_full, 4);
-      mbar_init(&sc.o_full, 1);
-      mbar_init(&sc.o_empty, 4);
-      mbar_init(&sc.final_bar, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&ctl->bm_full[b], 1);
+      mbar_init(&ctl->bm_empty[b], 9);  // eight softmax warps + the MMA issuer
+      mbar_init(&ctl->q_full[b], 1);
+      mbar_init(&ctl->q_empty[b], 1);
+      mbar_init(&ctl->s_full[b], 1);
+      mbar_init(&ctl->p_full[b], 8);
+      mbar_init(&ctl->pv_done[b], 1);
+      mbar_init(&ctl->o_full[b], 1);
+      mbar_init(&ctl->o_empty[b], 8);
+      mbar_init(&ctl->xbar[b], 8);
     }
+    for (int s = 0; s < 3; ++s) {
+      mbar_init(&ctl->k_full[s], 1);
+      mbar_init(&ctl->k_empty[s], 1);
+      mbar_init(&ctl->v_full[s], 1);
+      mbar_init(&ctl->v_empty[s], 1);
+    }
+    mbar_init(&ctl->final_bar, 1);
     ctl->abort.v = 0;
     fence_mbar_init();
   }
-  if (warp == 10) {
+  if (warp == 9) {
     tmem_alloc(&ctl->tmem_base, C::TMEM_COLS);
     tmem_relinquish();
   }
@@ -695,18 +732,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp < 8) {
     softmax_role<BS, D>(warp >> 2, args, ctl, tmem);
     __syncwarp();
-  } else {
-    if (warp < 10) {
-      load_role<BS, D>(warp - 8, &tmQ, &tmK, &tmV, args, smem, ctl);
-    } else {
-      if ((threadIdx.x & 31) == 0) mma_role<BS, D>(warp - 10, args, smem, ctl, tmem);
-      __syncwarp();
-    }
+  } else if (warp == 8) {
+    load_role<BS, D>(&tmQ, &tmK, &tmV, args, smem, ctl);
+  } else if (warp == 9) {
+    if ((threadIdx.x & 31) == 0) mma_role<BS, D>(args, smem, ctl, tmem);
+    __syncwarp();
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 10) {
+  if (warp == 9) {
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
   }
