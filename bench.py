@@ -54,6 +54,31 @@ KERNEL_DIR = os.path.join(ROOT, "block_sparse_attention_38_b200", "csrc")
 NCU_TRAFFIC = {}
 
 
+def replica_seed(w, rank: int) -> int:
+    """Seed of rank `rank`'s replica of workload w (rank 0 uses the workload's own seed)."""
+    return w.seed + 1000 * rank
+
+
+def max_over_ranks(values, world: int, device=None):
+    """Element-wise maximum of `values` over all ranks (identity for one rank).
+
+    Every rank calls it with the same number of values; the reduction runs on
+    the process group's backend (NCCL with device tensors, gloo on the CPU)."""
+    if world == 1:
+        return [float(v) for v in values]
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.cpu()]
+
+
+def whole_job_tflops(flops_per_rank: float, world: int, ms_per_step: float) -> float:
+    """Aggregate useful TFLOP/s of `world` replicas that each did flops_per_rank in ms_per_step."""
+    return flops_per_rank * world / (ms_per_step * 1e-3) / 1e12
+
+
 def useful_flops(w, nnz_all_heads: int) -> float:
     return 4.0 * w.block_size * w.block_size * w.d * nnz_all_heads * w.B
 
@@ -203,7 +228,7 @@ def run_ours(args, w, rank, world, local_rank):
     bsa.library()
 
     # Inputs: each rank its own replica (seed offset by rank).
-    q_h, k_h, v_h = workloads.make_qkv(w, seed=w.seed + 1000 * rank)
+    q_h, k_h, v_h = workloads.make_qkv(w, seed=replica_seed(w, rank))
     rp_np, ci_np = bsa.build_pattern_from(w.pattern)
     nnz = int(len(ci_np))
     flops = useful_flops(w, nnz)
@@ -286,16 +311,13 @@ def run_ours(args, w, rank, world, local_rank):
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1) / e_steps
 
-    t_max = torch.tensor([total_ms, e2e_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t_max, op=dist.ReduceOp.MAX)
-    total_ms, e2e_ms = float(t_max[0]), float(t_max[1])
+    total_ms, e2e_ms = max_over_ranks([total_ms, e2e_ms], world, device=dev)
     if rank != 0:
         return
 
     ms = total_ms / args.steps
-    value = flops * world / (ms * 1e-3) / 1e12
-    e2e_value = flops * world / (e2e_ms * 1e-3) / 1e12
+    value = whole_job_tflops(flops, world, ms)
+    e2e_value = whole_job_tflops(flops, world, e2e_ms)
     peaks, peak_src = load_peaks()
     peak_tc = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     peak_hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
