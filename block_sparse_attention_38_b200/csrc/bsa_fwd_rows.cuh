@@ -13,30 +13,29 @@
 // Sparse Attention with Log-Linear Complexity", section 3.3); the exponentials
 // of such blocks are not evaluated (membership is uniform over a warp).
 //
-// One persistent CTA per SM.  S and O are double-buffered in TMEM, so the MMA
-// issuer runs one step ahead of the softmax: while the softmax turns S(j)
-// into P(j), the tensor core computes S(j+1); then O += P(j) V(j) and S(j+2).
-// The next tile's first steps overlap the previous tile's epilogue the same
-// way.  Roles (384 threads):
-//   warps 0-3   softmax, columns 0-63 of every step (keys 0..63), and the
-//               epilogue of O columns [0, d/2)
-//   warps 4-7   the same for columns 64-127 and O columns [d/2, d)
-//   warp 8      tile schedule, per-tile block bitmaps, TMA loads of Q, K, V
-//   warp 9      tcgen05.mma issuer (and owner of the 512 TMEM columns)
-// The two softmax warpgroups cover the same 128 rows (TMEM lane quadrant
-// warp % 4); per step they exchange the row maximum of their halves through
-// shared memory (an mbarrier with bounded waits, not a hardware barrier, so
-// that a warpgroup giving up cannot leave the other waiting), so both use the
-// same running maximum; their partial sums are added at the end of the tile.
+// One persistent CTA per SM.  S is held in NS TMEM buffers and O in two, so
+// the MMA issuer runs NS - 1 steps ahead of the softmax: while the softmax
+// turns S(j) into P(j), the tensor core computes the next scores; then
+// O += P(j) V(j) and S(j+NS).  A tile's first steps overlap the previous
+// tile's epilogue the same way.  Roles (576 threads):
+//   warps 0-15  softmax: warpgroup q takes keys 32q..32q+31 of every step for
+//               all 128 rows (TMEM lane quadrant warp % 4) and O columns
+//               [q d/4, (q+1) d/4) in the epilogue
+//   warp 16     tile schedule, per-tile block bitmaps, TMA loads of Q, K, V
+//   warp 17     tcgen05.mma issuer (and owner of the 512 TMEM columns)
+// The four warps holding the same rows exchange their partial row maxima each
+// step through shared memory (an mbarrier with bounded waits, not a hardware
+// barrier, so that a warp giving up cannot leave the others waiting); their
+// partial sums are added at the end of the tile.
 //
-// TMEM columns: S(j) in [128 (j&1), +128); P(j) over the columns already
-// read: keys 0..63 at [128 (j&1), +32), keys 64..127 at [128 (j&1) + 64, +32);
-// O of tile t in [256 + d (t&1), +d).
+// TMEM columns: S(j) in [128 (j mod NS), +128); warpgroup q writes P of its
+// 32 keys over the first 16 of its own 32 score columns; O of tile t in
+// [128 NS + d (t&1), +d).
 //
 // Work split (`schedule`): tiles whose estimated cost (longest row plus one
 // step) exceeds half of a CTA's share -- the global rows of the local+global
-// pattern -- are dealt out one per CTA first; the remaining tiles are cut into
-// contiguous ranges that fill each CTA's leftover share.
+// pattern -- are dealt out one per CTA first; the other tiles go out in
+// round-robin rounds so that concurrent CTAs share K/V blocks in L2.
 #pragma once
 
 #include "bsa_common.cuh"
@@ -44,7 +43,9 @@
 namespace bsa {
 namespace rows {
 
-constexpr int kThreads = 384;
+constexpr int kSoftWG = 4;                 // softmax warpgroups; each takes 128 / kSoftWG keys of a step
+constexpr int kSoftWarps = 4 * kSoftWG;
+constexpr int kThreads = 32 * kSoftWarps + 64;  // + the producer warp and the MMA warp
 
 template <int BS, int D>
 struct Cfg {
@@ -62,9 +63,15 @@ struct Cfg {
   static constexpr int OFF_V = OFF_K + NKS * CH_BYTES;
   static constexpr int OFF_CTRL = OFF_V + NVS * CH_BYTES;
   static constexpr uint32_t TMEM_COLS = 512;
-  static constexpr uint32_t TMEM_O = 256;
+  // S buffers in TMEM: the MMA issuer runs NS - 1 steps ahead of the
+  // softmax.  Three fit beside two O accumulators for d = 64; for d = 128 the
+  // second O buffer (the next tile's PVs overlap this tile's epilogue) was
+  // measured to matter more than a third S buffer.
+  static constexpr int NS = D == 64 ? 3 : 2;
+  static constexpr uint32_t TMEM_O = NS * 128;   // O accumulators follow the S buffers
+  static constexpr int OB = 2;                   // tiles whose O fit side by side
   static_assert((Q_BYTES % 1024) == 0 && (CH_BYTES % 1024) == 0, "1024-byte aligned stages");
-  static_assert(TMEM_O + 2 * D <= TMEM_COLS, "TMEM layout");
+  static_assert(TMEM_O + OB * D <= TMEM_COLS, "TMEM layout");
   static_assert(TM == NK, "Q and K tiles share one slice-offset formula");
 };
 
@@ -92,16 +99,16 @@ struct Ctrl {
   uint64_t bm_full[2], bm_empty[2];
   uint64_t q_full[2], q_empty[2];
   uint64_t k_full[3], k_empty[3], v_full[3], v_empty[3];
-  uint64_t s_full[2], p_full[2], pv_done[2];
+  uint64_t s_full[3], p_full[3], pv_done[3];
   uint64_t o_full[2], o_empty[2];
-  uint64_t xbar[2];   // exchanges between the two softmax warpgroups
+  uint64_t xbar[2][4];  // [exchange parity][lane quadrant]: one warp of each softmax warpgroup
   uint64_t final_bar;
   long long tile[2];  // tile index of each bitmap buffer, -1 = no more work
   int n[2];           // union size (blocks) of each bitmap buffer
   Sched sched;
   uint32_t tmem_base;
   AbortFlag abort;
-  float red[2][2][128];      // [exchange parity][half][row]: partial row max or sum
+  float red[2][kSoftWG][128];  // [exchange parity][warpgroup][row]: partial row max or sum
   uint32_t bitmap[2][5 * kMaxBitmapWords];  // R block-row maps, then their union
 };
 
@@ -419,12 +426,12 @@ __device__ void mma_role(const FwdArgs& a, uint8_t* smem, Ctrl* ctl, uint32_t tm
     const uint32_t qb = q_uses & 1;
     if (!wait_bounded(&ctl->q_full[qb], (q_uses >> 1) & 1, &ctl->abort)) break;
     ++q_uses;
-    const uint32_t ob = o_tiles & 1;
+    const uint32_t ob = o_tiles % C::OB;
     const uint32_t t_o = tmem + C::TMEM_O + ob * D;
     const uint32_t q_tile = q_base + qb * C::Q_BYTES;
 
     auto issue_qk = [&](int j) -> bool {
-      const uint32_t sb = (gstep + j) & 1;
+      const uint32_t sb = (gstep + j) % C::NS;
       const uint32_t ks = k_cons % C::NKS;
       if (!wait_bounded(&ctl->k_full[ks], (k_cons / C::NKS) & 1, &ctl->abort)) return false;
       tc_fence_after();
@@ -444,20 +451,21 @@ __device__ void mma_role(const FwdArgs& a, uint8_t* smem, Ctrl* ctl, uint32_t tm
       return true;
     };
     auto issue_pv = [&](int j) -> bool {
-      const uint32_t gs = gstep + j, sb = gs & 1;
-      if (!wait_bounded(&ctl->p_full[sb], (gs >> 1) & 1, &ctl->abort)) return false;
+      const uint32_t gs = gstep + j, sb = gs % C::NS;
+      if (!wait_bounded(&ctl->p_full[sb], (gs / C::NS) & 1, &ctl->abort)) return false;
       const uint32_t vs = v_cons % C::NVS;
       if (!wait_bounded(&ctl->v_full[vs], (v_cons / C::NVS) & 1, &ctl->abort)) return false;
-      if (j == 0 && o_tiles >= 2 &&
-          !wait_bounded(&ctl->o_empty[ob], ((o_tiles - 2) >> 1) & 1, &ctl->abort))
+      if (j == 0 && o_tiles >= C::OB &&
+          !wait_bounded(&ctl->o_empty[ob], ((o_tiles - C::OB) / C::OB) & 1, &ctl->abort))
         return false;
       tc_fence_after();
       const uint64_t bd0 = sdesc_sw128(v_base + vs * C::CH_BYTES, C::NK * 128, 1024);
       const uint32_t a0 = tmem + sb * 128;
 #pragma unroll
       for (int kk = 0; kk < C::NK / 16; ++kk) {
-        // P of keys 16kk..16kk+15: columns 8kk (keys < 64) or 64 + 8(kk-4) (keys >= 64).
-        const uint32_t a_col = kk < 4 ? kk * 8 : 64 + (kk - 4) * 8;
+        // P of keys 16kk..16kk+15: warpgroup kk/2 packs its 32 keys into the
+        // first 16 of its 32 score columns.
+        const uint32_t a_col = (kk >> 1) * 32 + (kk & 1) * 8;
         umma_bf16_ts(t_o, a0 + a_col, bd0 + ((kk * 16 * 128) >> 4), kIdescPV,
                      (j > 0 || kk > 0) ? 1u : 0u);
       }
@@ -468,8 +476,10 @@ __device__ void mma_role(const FwdArgs& a, uint8_t* smem, Ctrl* ctl, uint32_t tm
       return true;
     };
 
-    ok = issue_qk(0) && (steps < 2 || issue_qk(1));
-    for (int j = 0; ok && j < steps; ++j) ok = issue_pv(j) && (j + 2 >= steps || issue_qk(j + 2));
+    ok = issue_qk(0);
+    for (int j = 1; ok && j < C::NS && j < steps; ++j) ok = issue_qk(j);
+    for (int j = 0; ok && j < steps; ++j)
+      ok = issue_pv(j) && (j + C::NS >= steps || issue_qk(j + C::NS));
     gstep += steps;
     ++o_tiles;
   }
@@ -479,13 +489,15 @@ __device__ void mma_role(const FwdArgs& a, uint8_t* smem, Ctrl* ctl, uint32_t tm
 }
 
 // ------------------------------------------------------------ softmax warps
-// Warpgroup `half` handles keys 64*half .. 64*half+63 of every step (two
-// groups of 32 TMEM columns) for all 128 rows, and O columns
-// [half*d/2, (half+1)*d/2) in the epilogue.
+// Warpgroup `qt` handles keys 32 qt .. 32 qt + 31 of every step (one group of
+// 32 TMEM columns) for all 128 rows, and O columns [qt d/4, (qt+1) d/4) in
+// the epilogue.  The kSoftWG warps that hold the same rows (one per
+// warpgroup, TMEM lane quadrant wq) exchange their partial row maxima each
+// step and their partial sums at the end of a tile.
 template <int BS, int D>
-__device__ void softmax_role(int half, const FwdArgs& a, Ctrl* ctl, uint32_t tmem) {
+__device__ void softmax_role(int qt, const FwdArgs& a, Ctrl* ctl, uint32_t tmem) {
   using C = Cfg<BS, D>;
-  constexpr int HD = D / 2;                    // O columns of this warpgroup
+  constexpr int QD = D / kSoftWG;              // O columns of this warpgroup (16 or 32)
   const int wq = (threadIdx.x >> 5) & 3;       // TMEM lane quadrant
   const int lane = threadIdx.x & 31;
   const int row = wq * 32 + lane;              // query row of the tile
@@ -494,17 +506,18 @@ __device__ void softmax_role(int half, const FwdArgs& a, Ctrl* ctl, uint32_t tme
   const uint32_t t_lane = static_cast<uint32_t>(wq * 32) << 16;
   const float sl2 = a.scale_log2;
   constexpr float kNegInf = -INFINITY;
+  const int b_mine = (qt * 32) / BS;           // block of the step holding this group
+  const int c0 = (qt * 32) % BS;               // first column of the group inside its block
   uint32_t gstep = 0, o_tiles = 0, n_ex = 0;
-  // Both warpgroups have written their values for exchange number n_ex:
-  // every warp arrives on xbar[n_ex & 1] (eight warps in all) and waits for
-  // the phase (bounded).  Values live in buffer n_ex & 1, so the next write
-  // to a buffer comes after the other warpgroup has passed the exchange that
-  // read it.
+  // The warps sharing these rows have written their values for exchange
+  // n_ex: each arrives on xbar[n_ex & 1][wq] (kSoftWG arrivals complete it)
+  // and waits for the phase (bounded).  Values live in buffer n_ex & 1, so
+  // the next write to a buffer comes after every partner has passed the
+  // exchange that read it.
   auto exchange = [&]() -> bool {
     __syncwarp();
-    if (lane == 0) mbar_arrive(&ctl->xbar[n_ex & 1]);
-    const bool ok = warp_wait(&ctl->xbar[n_ex & 1], (n_ex >> 1) & 1, &ctl->abort);
-    return ok;
+    if (lane == 0) mbar_arrive(&ctl->xbar[n_ex & 1][wq]);
+    return warp_wait(&ctl->xbar[n_ex & 1][wq], (n_ex >> 1) & 1, &ctl->abort);
   };
 
   for (int t = 0;; ++t) {
@@ -521,66 +534,56 @@ __device__ void softmax_role(int half, const FwdArgs& a, Ctrl* ctl, uint32_t tme
     const bool row_ok = r_sub < a.M;
     const int steps = (n + C::BPS - 1) / C::BPS;
     const long long qtok = static_cast<long long>(g) * C::TM + row;
-    uint4* orow = reinterpret_cast<uint4*>(a.O + (bh * a.N + qtok) * D + half * HD);
+    uint4* orow = reinterpret_cast<uint4*>(a.O + (bh * a.N + qtok) * D + qt * QD);
 
     if (n == 0) {
       if (row_ok) {
 #pragma unroll
-        for (int c = 0; c < HD / 8; ++c) orow[c] = make_uint4(0u, 0u, 0u, 0u);
-        if (half == 0) a.LSE[bh * a.N + qtok] = kNegInf;
+        for (int c = 0; c < QD / 8; ++c) orow[c] = make_uint4(0u, 0u, 0u, 0u);
+        if (qt == 0) a.LSE[bh * a.N + qtok] = kNegInf;
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&ctl->bm_empty[buf]);
       continue;
     }
 
-    float m_used = kNegInf;  // running max, log2 units of the scaled score (same in both halves)
-    float l = 0.f;           // this half's running sum of 2^(s - m_used)
+    float m_used = kNegInf;  // running max, log2 units of the scaled score (same in every warpgroup)
+    float l = 0.f;           // this warpgroup's running sum of 2^(s - m_used)
+    const uint32_t ob = o_tiles % C::OB;
     BitIter it(bm + C::R * a.W, a.W);
     for (int j = 0; j < steps; ++j) {
-      const uint32_t gs = gstep + j, sb = gs & 1;
-      // This half's two 32-column groups: vmask bit i = the row holds the
-      // block of group i, dmask bit i = that block is its causal diagonal.
-      uint32_t vmask = 0, dmask = 0;
+      const uint32_t gs = gstep + j, sb = gs % C::NS;
+      bool valid = false, diag = false;  // this row holds the group's block / it is the diagonal
 #pragma unroll
       for (int b = 0; b < C::BPS; ++b) {
         const int jb = it.next();
-#pragma unroll
-        for (int i = 0; i < 2; ++i) {
-          if ((2 * half + i) * 32 / BS != b) continue;
-          if (row_ok && jb >= 0 && ((mine[jb >> 5] >> (jb & 31)) & 1u)) vmask |= 1u << i;
-          if (a.causal && jb == r_sub) dmask |= 1u << i;
-        }
+        if (b != b_mine) continue;
+        valid = row_ok && jb >= 0 && ((mine[jb >> 5] >> (jb & 31)) & 1u);
+        diag = a.causal && jb == r_sub;
       }
-      if (!warp_wait(&ctl->s_full[sb], (gs >> 1) & 1, &ctl->abort)) return;
+      if (!warp_wait(&ctl->s_full[sb], (gs / C::NS) & 1, &ctl->abort)) return;
       tc_fence_after();
-      const uint32_t t_s = tmem + t_lane + sb * 128 + half * 64;
-      uint32_t u[64];
+      const uint32_t t_s = tmem + t_lane + sb * 128 + qt * 32;
+      uint32_t u[32];
       float pmax = kNegInf;
-      if (vmask != 0) {  // uniform over the warp
-        tmem_ld32(t_s, *reinterpret_cast<uint32_t(*)[32]>(&u[0]));
-        tmem_ld32(t_s + 32, *reinterpret_cast<uint32_t(*)[32]>(&u[32]));
+      if (valid) {  // uniform over the warp
+        tmem_ld32(t_s, u);
         tmem_wait_ld();
-        reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&u[0]));
-        reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&u[32]));
+        reg_fence32(u);
 #pragma unroll
-        for (int i = 0; i < 2; ++i) {
-          if (!((vmask >> i) & 1u)) continue;
-          const bool diag = (dmask >> i) & 1u;
-          const int c0 = ((2 * half + i) * 32) % BS;  // first column of the group inside its block
-#pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            float v = __uint_as_float(u[i * 32 + c]) * sl2;
-            if (diag && c0 + c > qq) v = kNegInf;  // key after the query (diagonal block only)
-            u[i * 32 + c] = __float_as_uint(v);
-            pmax = fmaxf(pmax, v);
-          }
+        for (int c = 0; c < 32; ++c) {
+          float v = __uint_as_float(u[c]) * sl2;
+          if (diag && c0 + c > qq) v = kNegInf;  // key after the query (diagonal block only)
+          u[c] = __float_as_uint(v);
+          pmax = fmaxf(pmax, v);
         }
       }
-      // Row maximum over both halves.
-      ctl->red[n_ex & 1][half][row] = pmax;
+      // Row maximum over all warpgroups.
+      ctl->red[n_ex & 1][qt][row] = pmax;
       if (!exchange()) return;
-      const float mx = fmaxf(pmax, ctl->red[n_ex & 1][half ^ 1][row]);
+      float mx = kNegInf;
+#pragma unroll
+      for (int o = 0; o < kSoftWG; ++o) mx = fmaxf(mx, ctl->red[n_ex & 1][o][row]);
       ++n_ex;
 
       // Lazy rescale: the running maximum moves only when the step's maximum
@@ -597,89 +600,80 @@ __device__ void softmax_role(int half, const FwdArgs& a, Ctrl* ctl, uint32_t tme
       if (__any_sync(0xffffffffu, need_rescale)) {
         // O must hold every PV up to the previous step.
         const uint32_t pg = gs - 1;
-        if (!warp_wait(&ctl->pv_done[pg & 1], (pg >> 1) & 1, &ctl->abort)) return;
+        if (!warp_wait(&ctl->pv_done[pg % C::NS], (pg / C::NS) & 1, &ctl->abort)) return;
         tc_fence_after();
-        const uint32_t t_o = tmem + t_lane + C::TMEM_O + (o_tiles & 1) * D + half * HD;
-#pragma unroll 1
-        for (int c = 0; c < HD / 32; ++c) {
-          uint32_t w[32];
-          tmem_ld32(t_o + c * 32, w);
-          tmem_wait_ld();
-          reg_fence32(w);
+        const uint32_t t_o = tmem + t_lane + C::TMEM_O + ob * D + qt * QD;
+        uint32_t w[32];
+        if constexpr (QD == 32) tmem_ld32(t_o, w);
+        else tmem_ld16(t_o, *reinterpret_cast<uint32_t(*)[16]>(&w[0]));
+        tmem_wait_ld();
+        reg_fence32(w);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) w[i] = __float_as_uint(__uint_as_float(w[i]) * factor);
-          tmem_st32(t_o + c * 32, w);
-        }
+        for (int i = 0; i < QD; ++i) w[i] = __float_as_uint(__uint_as_float(w[i]) * factor);
+        if constexpr (QD == 32) tmem_st32(t_o, w);
+        else tmem_st16(t_o, *reinterpret_cast<uint32_t(*)[16]>(&w[0]));
       }
       l *= factor;
 
-      uint32_t pk[32];
-      if (vmask != 0) {
+      uint32_t pk[16];
+      if (valid) {
         const float mu = m_used == kNegInf ? 0.f : m_used;
         float rs = 0.f;
 #pragma unroll
-        for (int i = 0; i < 2; ++i) {
-          const bool on = (vmask >> i) & 1u;
-#pragma unroll
-          for (int c = 0; c < 32; c += 2) {
-            float p0 = 0.f, p1 = 0.f;
-            if (on) {
-              p0 = ex2_approx(__uint_as_float(u[i * 32 + c]) - mu);
-              p1 = ex2_approx(__uint_as_float(u[i * 32 + c + 1]) - mu);
-              rs += p0;
-              rs += p1;
-            }
-            pk[i * 16 + c / 2] = pack_bf16x2(p0, p1);
-          }
+        for (int c = 0; c < 32; c += 2) {
+          const float p0 = ex2_approx(__uint_as_float(u[c]) - mu);
+          const float p1 = ex2_approx(__uint_as_float(u[c + 1]) - mu);
+          rs += p0;
+          rs += p1;
+          pk[c / 2] = pack_bf16x2(p0, p1);
         }
         l += rs;
       } else {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) pk[i] = 0u;
+        for (int i = 0; i < 16; ++i) pk[i] = 0u;
       }
-      tmem_st32(tmem + t_lane + sb * 128 + half * 64, pk);  // P columns of this half
+      tmem_st16(t_s, pk);  // P of this group's 32 keys, over its first 16 columns
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&ctl->p_full[sb]);
     }
 
-    // Epilogue: O / l in bf16 (this half's columns) and LSE = (m + log2 l) ln 2.
-    ctl->red[n_ex & 1][half][row] = l;
+    // Epilogue: O / l in bf16 (this warpgroup's columns) and LSE = (m + log2 l) ln 2.
+    ctl->red[n_ex & 1][qt][row] = l;
     if (!exchange()) return;
-    const float lt = l + ctl->red[n_ex & 1][half ^ 1][row];
+    float lt = 0.f;
+#pragma unroll
+    for (int o = 0; o < kSoftWG; ++o) lt += ctl->red[n_ex & 1][o][row];
     ++n_ex;
-    const uint32_t ob = o_tiles & 1;
-    if (!warp_wait(&ctl->o_full[ob], (o_tiles >> 1) & 1, &ctl->abort)) return;
+    if (!warp_wait(&ctl->o_full[ob], (o_tiles / C::OB) & 1, &ctl->abort)) return;
     tc_fence_after();
     const float inv = lt > 0.f ? 1.f / lt : 0.f;
-    const uint32_t t_o = tmem + t_lane + C::TMEM_O + ob * D + half * HD;
-#pragma unroll 1
-    for (int c = 0; c < HD / 32; ++c) {
-      uint32_t w[32];
-      tmem_ld32(t_o + c * 32, w);
-      tmem_wait_ld();
-      reg_fence32(w);
-      if (row_ok) {
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          uint4 v;
-          v.x = pack_bf16x2(__uint_as_float(w[q * 8 + 0]) * inv, __uint_as_float(w[q * 8 + 1]) * inv);
-          v.y = pack_bf16x2(__uint_as_float(w[q * 8 + 2]) * inv, __uint_as_float(w[q * 8 + 3]) * inv);
-          v.z = pack_bf16x2(__uint_as_float(w[q * 8 + 4]) * inv, __uint_as_float(w[q * 8 + 5]) * inv);
-          v.w = pack_bf16x2(__uint_as_float(w[q * 8 + 6]) * inv, __uint_as_float(w[q * 8 + 7]) * inv);
-          orow[c * 4 + q] = v;
-        }
-      }
-    }
+    const uint32_t t_o = tmem + t_lane + C::TMEM_O + ob * D + qt * QD;
+    uint32_t w[32];
+    if constexpr (QD == 32) tmem_ld32(t_o, w);
+    else tmem_ld16(t_o, *reinterpret_cast<uint32_t(*)[16]>(&w[0]));
+    tmem_wait_ld();
+    reg_fence32(w);
     tc_fence_before();
     __syncwarp();
     if (lane == 0) {
       mbar_arrive(&ctl->o_empty[ob]);
       mbar_arrive(&ctl->bm_empty[buf]);
     }
-    if (half == 0 && row_ok)
-      a.LSE[bh * a.N + qtok] = lt > 0.f ? (m_used + __log2f(lt)) * 0.69314718055994531f : kNegInf;
+    if (row_ok) {
+#pragma unroll
+      for (int q = 0; q < QD / 8; ++q) {
+        uint4 v;
+        v.x = pack_bf16x2(__uint_as_float(w[q * 8 + 0]) * inv, __uint_as_float(w[q * 8 + 1]) * inv);
+        v.y = pack_bf16x2(__uint_as_float(w[q * 8 + 2]) * inv, __uint_as_float(w[q * 8 + 3]) * inv);
+        v.z = pack_bf16x2(__uint_as_float(w[q * 8 + 4]) * inv, __uint_as_float(w[q * 8 + 5]) * inv);
+        v.w = pack_bf16x2(__uint_as_float(w[q * 8 + 6]) * inv, __uint_as_float(w[q * 8 + 7]) * inv);
+        orow[q] = v;
+      }
+      if (qt == 0)
+        a.LSE[bh * a.N + qtok] = lt > 0.f ? (m_used + __log2f(lt)) * 0.69314718055994531f : kNegInf;
+    }
     gstep += steps;
     ++o_tiles;
   }
@@ -699,17 +693,18 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     for (int b = 0; b < 2; ++b) {
       mbar_init(&ctl->bm_full[b], 1);
-      mbar_init(&ctl->bm_empty[b], 9);  // eight softmax warps + the MMA issuer
+      mbar_init(&ctl->bm_empty[b], kSoftWarps + 1);  // the softmax warps + the MMA issuer
       mbar_init(&ctl->q_full[b], 1);
       mbar_init(&ctl->q_empty[b], 1);
-      mbar_init(&ctl->s_full[b], 1);
-      mbar_init(&ctl->p_full[b], 8);
-      mbar_init(&ctl->pv_done[b], 1);
+
       mbar_init(&ctl->o_full[b], 1);
-      mbar_init(&ctl->o_empty[b], 8);
-      mbar_init(&ctl->xbar[b], 8);
+      mbar_init(&ctl->o_empty[b], kSoftWarps);
+      for (int q = 0; q < 4; ++q) mbar_init(&ctl->xbar[b][q], kSoftWG);
     }
     for (int s = 0; s < 3; ++s) {
+      mbar_init(&ctl->s_full[s], 1);
+      mbar_init(&ctl->p_full[s], kSoftWarps);
+      mbar_init(&ctl->pv_done[s], 1);
       mbar_init(&ctl->k_full[s], 1);
       mbar_init(&ctl->k_empty[s], 1);
       mbar_init(&ctl->v_full[s], 1);
@@ -719,7 +714,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     ctl->abort.v = 0;
     fence_mbar_init();
   }
-  if (warp == 9) {
+  if (warp == kSoftWarps + 1) {
     tmem_alloc(&ctl->tmem_base, C::TMEM_COLS);
     tmem_relinquish();
   }
@@ -729,19 +724,19 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = ctl->tmem_base;
 
-  if (warp < 8) {
+  if (warp < kSoftWarps) {
     softmax_role<BS, D>(warp >> 2, args, ctl, tmem);
     __syncwarp();
-  } else if (warp == 8) {
+  } else if (warp == kSoftWarps) {
     load_role<BS, D>(&tmQ, &tmK, &tmV, args, smem, ctl);
-  } else if (warp == 9) {
+  } else if (warp == kSoftWarps + 1) {
     if ((threadIdx.x & 31) == 0) mma_role<BS, D>(args, smem, ctl, tmem);
     __syncwarp();
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == kSoftWarps + 1) {
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
   }

@@ -145,6 +145,24 @@ def test_random_patterns(shape, causal):
     _compare(O, L, Or, Lr, str(shape))
 
 
+@pytest.mark.parametrize("scale", [-0.2, 0.0, 0.7])
+@pytest.mark.parametrize("shape", [(1, 2, 256, 64, 32), (1, 2, 384, 128, 64), (1, 2, 512, 128, 128)],
+                         ids=lambda s: "B{}H{}N{}d{}bs{}".format(*s))
+def test_negative_zero_and_large_scale(shape, scale):
+    # the kernel is specialised on the sign of the scale (maximum or minimum
+    # of the raw scores); scale 0 gives uniform weights over the allowed keys
+    B, H, N, d, bs = shape
+    M = N // bs
+    rng = np.random.default_rng(int(abs(scale) * 1000) + N)
+    q, k, v = workloads.make_qkv_shape(B, H, N, d, seed=int(rng.integers(1 << 30)))
+    for causal in (False, True):
+        rp, ci = _random_csr(rng, H, M, 0.5, causal, shuffle=False, dup=False, empty_rows=1)
+        O, L = _run_gpu(q, k, v, rp, ci, bs, scale, causal)
+        assert bsa.device_status(clear=True) == 0
+        Or, Lr, _ = oracle.forward(q, k, v, rp, ci, bs, scale, causal)
+        _compare(O, L, Or, Lr, f"{shape} scale={scale} causal={causal}")
+
+
 @pytest.mark.parametrize("d", [64, 128])
 @pytest.mark.parametrize("bs", [32, 64, 128])
 def test_many_tiles_per_cta_varying_row_lengths(bs, d):
