@@ -52,8 +52,7 @@ KERNEL_DIR = os.path.join(ROOT, "block_sparse_attention_38_b200", "csrc")
 # workload, valid only for the kernel sources whose sha256 prefix is given
 # (profiles/ holds the capture summaries).
 NCU_TRAFFIC = {
-    "loglinear_4k": (25391872, "5b9e319b03f46632"),
-    "local_global_8k": (290147584 + 47099904, "5b9e319b03f46632"),
+    "loglinear_4k": (25392640, "cab8e846fd2d847e"),
 }
 
 
