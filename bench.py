@@ -53,6 +53,9 @@ KERNEL_DIR = os.path.join(ROOT, "block_sparse_attention_38_b200", "csrc")
 # (profiles/ holds the capture summaries).
 NCU_TRAFFIC = {
     "loglinear_4k": (25392640, "cab8e846fd2d847e"),
+    "local_global_8k": (293797376 + 48656896, "cab8e846fd2d847e"),
+    "bernoulli_4k": (201550592 + 51967488, "cab8e846fd2d847e"),
+    "causal_loglinear_32k": (806639360 + 254766848, "cab8e846fd2d847e"),
 }
 
 

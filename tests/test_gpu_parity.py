@@ -189,6 +189,24 @@ def test_many_tiles_per_cta_varying_row_lengths(bs, d):
     _compare(O.reshape(-1, d)[rows_s], L.reshape(-1)[rows_s], Or, Lr, f"bs={bs} d={d}")
 
 
+@pytest.mark.parametrize("bs,d", [(64, 128), (32, 64)])
+def test_many_global_rows_exercise_the_heavy_tile_schedule(bs, d):
+    # local+global with six full rows per head: tiles holding a global row
+    # cost many times the others, so they are dealt out one per CTA first and
+    # those CTAs sit out the first rounds of the other tiles; every output row
+    # is compared
+    B, H, N = 2, 4, 4096
+    M = N // bs
+    desc = workloads.PatternDesc(kind=workloads.LOCAL_GLOBAL, M=M, H=H, local_radius=2,
+                                 anchors=(0, 5, M // 3, M // 2, M - 7, M - 1))
+    rp, ci = patterns.csr(desc)
+    q, k, v = workloads.make_qkv_shape(B, H, N, d, seed=bs + 7 * d, key_scale_max=3.0)
+    O, L = _run_gpu(q, k, v, rp, ci, bs, 1.0 / math.sqrt(d), False)
+    assert bsa.device_status(clear=True) == 0
+    Or, Lr, _ = oracle.forward(q, k, v, rp, ci, bs, 1.0 / math.sqrt(d), False)
+    _compare(O, L, Or, Lr, f"local_global bs={bs} d={d}")
+
+
 def test_all_rows_empty():
     B, H, N, d, bs = 1, 2, 256, 64, 32
     q, k, v = workloads.make_qkv_shape(B, H, N, d, seed=5)
