@@ -40,6 +40,8 @@ STATUS_NAMES = {OK: "BSA_OK", ERR_INVALID_ARG: "BSA_ERR_INVALID_ARG",
 LOGLINEAR = 0
 LOCAL_GLOBAL = 1
 BERNOULLI = 2
+SLIDING_WINDOW = 3
+BIGBIRD = 4
 
 # device status bits
 STATUS_TIMEOUT = 0x1
@@ -57,7 +59,8 @@ class _Desc(ctypes.Structure):
     _fields_ = [("kind", ctypes.c_int32), ("M", ctypes.c_int32), ("H", ctypes.c_int32),
                 ("local_radius", ctypes.c_int32), ("log_kmax", ctypes.c_int32),
                 ("n_anchors", ctypes.c_int32), ("anchors", ctypes.POINTER(ctypes.c_int32)),
-                ("p", ctypes.c_double), ("seed", ctypes.c_uint64), ("causal", ctypes.c_int32)]
+                ("p", ctypes.c_double), ("seed", ctypes.c_uint64), ("causal", ctypes.c_int32),
+                ("dilation", ctypes.c_int32), ("num_random", ctypes.c_int32)]
 
 
 _lib = None
@@ -96,7 +99,8 @@ def _check(code: int, what: str) -> None:
 
 def build_pattern(kind: int, M: int, H: int, local_radius: int = 1, log_kmax: int = 0,
                   anchors: Sequence[int] = (), p: float = 0.0, seed: int = 0,
-                  causal: bool = False) -> Tuple[np.ndarray, np.ndarray]:
+                  causal: bool = False, dilation: int = 1,
+                  num_random: int = 0) -> Tuple[np.ndarray, np.ndarray]:
     """Block-CSR of a pattern, built on the host by bsa_build_pattern.
 
     Returns (row_ptr int32 [H*M+1], col_idx int32 [nnz]) as numpy arrays.
@@ -105,7 +109,8 @@ def build_pattern(kind: int, M: int, H: int, local_radius: int = 1, log_kmax: in
     anc = np.ascontiguousarray(np.asarray(anchors, dtype=np.int32).reshape(-1))
     d = _Desc(int(kind), int(M), int(H), int(local_radius), int(log_kmax), int(anc.size),
               anc.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)) if anc.size else None,
-              float(p), int(seed) & ((1 << 64) - 1), int(bool(causal)))
+              float(p), int(seed) & ((1 << 64) - 1), int(bool(causal)), int(dilation),
+              int(num_random))
     nnz = ctypes.c_int64(0)
     _check(lib.bsa_build_pattern(ctypes.byref(d), None, None, 0, ctypes.byref(nnz)),
            "bsa_build_pattern")
@@ -119,7 +124,8 @@ def build_pattern(kind: int, M: int, H: int, local_radius: int = 1, log_kmax: in
 def build_pattern_from(desc) -> Tuple[np.ndarray, np.ndarray]:
     """build_pattern for any object with the bsa_pattern_desc field names."""
     return build_pattern(desc.kind, desc.M, desc.H, desc.local_radius, desc.log_kmax,
-                         desc.anchors, desc.p, desc.seed, desc.causal)
+                         desc.anchors, desc.p, desc.seed, desc.causal,
+                         getattr(desc, "dilation", 1), getattr(desc, "num_random", 0))
 
 
 def validate_pattern(row_ptr: np.ndarray, col_idx: np.ndarray, H: int, M: int,

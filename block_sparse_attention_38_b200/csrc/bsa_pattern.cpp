@@ -34,6 +34,15 @@ inline bool bernoulli_keep(const bsa_pattern_desc& d, int64_t h, int64_t i, int6
   return u < d.p;
 }
 
+// BigBird random column r of block row i, head h (draws with replacement).
+inline int32_t bigbird_column(const bsa_pattern_desc& d, int64_t h, int64_t i, int64_t r) {
+  const uint64_t key = static_cast<uint64_t>((h * d.M + i) * d.num_random + r);
+  const uint64_t top53 = splitmix64_at(d.seed, key + 1) >> 11;
+  const double u = static_cast<double>(top53) * (1.0 / 9007199254740992.0);  // 2^-53
+  const int64_t j = static_cast<int64_t>(u * d.M);
+  return static_cast<int32_t>(j < d.M ? j : d.M - 1);
+}
+
 // Appends the columns of block row i (head h) to out, ascending and distinct.
 void row_columns(const bsa_pattern_desc& d, int32_t h, int32_t i, std::vector<int32_t>& out,
                  std::vector<int32_t>& tmp) {
@@ -70,6 +79,27 @@ void row_columns(const bsa_pattern_desc& d, int32_t h, int32_t i, std::vector<in
         if (bernoulli_keep(d, h, i, j)) tmp.push_back(j);
       break;
     }
+    case BSA_SLIDING_WINDOW: {
+      const int64_t lo = std::max<int64_t>(0, int64_t(i) - d.local_radius);
+      const int64_t hi = std::min<int64_t>(M - 1, int64_t(i) + d.local_radius);
+      for (int64_t j = lo; j <= hi; ++j)
+        if ((int64_t(i) - j) % d.dilation == 0) tmp.push_back(static_cast<int32_t>(j));
+      break;
+    }
+    case BSA_BIGBIRD: {
+      bool global_row = false;
+      for (int32_t a = 0; a < d.n_anchors; ++a) global_row |= (d.anchors[a] == i);
+      if (global_row) {
+        for (int32_t j = 0; j < M; ++j) tmp.push_back(j);
+      } else {
+        const int64_t lo = std::max<int64_t>(0, int64_t(i) - d.local_radius);
+        const int64_t hi = std::min<int64_t>(M - 1, int64_t(i) + d.local_radius);
+        for (int64_t j = lo; j <= hi; ++j) tmp.push_back(static_cast<int32_t>(j));
+        for (int32_t a = 0; a < d.n_anchors; ++a) tmp.push_back(d.anchors[a]);
+        for (int32_t r = 0; r < d.num_random; ++r) tmp.push_back(bigbird_column(d, h, i, r));
+      }
+      break;
+    }
     default:
       break;
   }
@@ -85,13 +115,14 @@ void row_columns(const bsa_pattern_desc& d, int32_t h, int32_t i, std::vector<in
 bool desc_ok(const bsa_pattern_desc* d) {
   if (!d) return false;
   if (d->M < 1 || d->H < 1) return false;
-  if (d->kind != BSA_LOGLINEAR && d->kind != BSA_LOCAL_GLOBAL && d->kind != BSA_BERNOULLI)
-    return false;
+  if (d->kind < BSA_LOGLINEAR || d->kind > BSA_BIGBIRD) return false;
   if (d->local_radius < 0) return false;
   if (d->kind == BSA_LOGLINEAR && (d->log_kmax < 0 || d->log_kmax > 30)) return false;
   if (d->kind == BSA_BERNOULLI && !(d->p >= 0.0 && d->p <= 1.0)) return false;
   if (d->n_anchors < 0 || (d->n_anchors > 0 && d->anchors == nullptr)) return false;
   if (d->causal != 0 && d->causal != 1) return false;
+  if (d->kind == BSA_SLIDING_WINDOW && d->dilation < 1) return false;
+  if (d->kind == BSA_BIGBIRD && d->num_random < 0) return false;
   return true;
 }
 
@@ -105,8 +136,9 @@ extern "C" int bsa_build_pattern(const bsa_pattern_desc* desc, int32_t* row_ptr,
   const int64_t rows = int64_t(d.H) * d.M;
   if (rows + 1 > INT32_MAX) return BSA_ERR_INVALID_ARG;
 
-  // Heads repeat for the deterministic kinds; Bernoulli draws per head.
-  const int32_t distinct_heads = (d.kind == BSA_BERNOULLI) ? d.H : 1;
+  // Heads repeat for the deterministic kinds; Bernoulli and BigBird draw per head.
+  const bool per_head = d.kind == BSA_BERNOULLI || (d.kind == BSA_BIGBIRD && d.num_random > 0);
+  const int32_t distinct_heads = per_head ? d.H : 1;
   std::vector<int32_t> cols, tmp;
   std::vector<int64_t> head_ptr;  // row offsets inside cols for the distinct heads
   head_ptr.reserve(size_t(distinct_heads) * d.M + 1);
@@ -160,4 +192,4 @@ extern "C" int bsa_validate_pattern(const int32_t* row_ptr, const int32_t* col_i
   return BSA_OK;
 }
 
-extern "C" int bsa_version(void) { return 100; }
+extern "C" int bsa_version(void) { return 101; }

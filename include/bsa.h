@@ -55,7 +55,21 @@ typedef enum {
    * with probability p, drawn from the counter-based SplitMix64 stream of
    * `seed` (output number key+1, key = (h*M + i)*M + j, u = top 53 bits /
    * 2^53, kept iff u < p); the diagonal is always kept. */
-  BSA_BERNOULLI = 2
+  BSA_BERNOULLI = 2,
+  /* SparseFlashAttention article, "sparse pattern configuration examples"
+   * (sliding_window: window and dilation "like a dilated convolution"),
+   * taken at block level: column j is kept when |i-j| <= local_radius and
+   * (i-j) is a multiple of `dilation` (the diagonal always is). */
+  BSA_SLIDING_WINDOW = 3,
+  /* SparseFlashAttention article, same examples (bigbird: random blocks,
+   * block size, global tokens), with the three kinds of connections that
+   * "Block Sparse Attention with Log-Linear Complexity", section 2.2, lists for
+   * BigBird: a local window (|i-j| <= local_radius), global blocks (anchors:
+   * full rows and full columns, as for BSA_LOCAL_GLOBAL) and `num_random`
+   * random columns per (h, i): draw r = 0..num_random-1 takes output number
+   * key+1 of the SplitMix64 stream of `seed` with key = (h*M + i)*num_random + r,
+   * u = top 53 bits / 2^53, column floor(u*M); repeats merge. */
+  BSA_BIGBIRD = 4
 } bsa_kind;
 
 /* Pattern description (caller-owned; anchors points to n_anchors ints). */
@@ -71,6 +85,8 @@ typedef struct {
   double p;              /* BERNOULLI keep probability in [0, 1] */
   uint64_t seed;         /* BERNOULLI stream seed */
   int32_t causal;        /* 0 or 1: keep only columns j <= i */
+  int32_t dilation;      /* SLIDING_WINDOW: keep j with (i-j) % dilation == 0, >= 1 */
+  int32_t num_random;    /* BIGBIRD: random columns drawn per block row, >= 0 */
 } bsa_pattern_desc;
 
 /*
@@ -85,7 +101,9 @@ typedef struct {
  * Returns BSA_ERR_INVALID_ARG for a null desc/nnz_out, M < 1, H < 1, an
  * unknown kind, a negative radius, log_kmax outside [0, 30], p outside
  * [0, 1], n_anchors < 0 or anchors == NULL with n_anchors > 0, causal not
- * 0/1, or an nnz that does not fit int32.
+ * 0/1, dilation < 1 (SLIDING_WINDOW), num_random < 0 (BIGBIRD), or an nnz
+ * that does not fit int32.  BERNOULLI and BIGBIRD draw every head on its
+ * own; the other kinds repeat one head's rows.
  */
 int bsa_build_pattern(const bsa_pattern_desc* desc, int32_t* row_ptr, int32_t* col_idx,
                       int64_t cap, int64_t* nnz_out);

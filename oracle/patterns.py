@@ -93,6 +93,38 @@ def bernoulli_cols(h: int, i: int, M: int, p: float, seed: int,
     return keep
 
 
+def sliding_window_cols(i: int, M: int, w: int, dilation: int,
+                        causal: bool = False) -> List[int]:
+    """Dilated sliding window at block level (the SparseFlashAttention article's
+    sliding_window example): |i - j| <= w and (i - j) a multiple of the dilation."""
+    keep = [j for j in range(max(0, i - w), min(M - 1, i + w) + 1)
+            if (i - j) % dilation == 0 and (not causal or j <= i)]
+    return keep
+
+
+def bigbird_random_col(seed: int, h: int, i: int, r: int, M: int, num_random: int) -> int:
+    """Random column r of block row i, head h: output key+1 of the SplitMix64
+    stream at `seed`, key = (h*M + i)*num_random + r, scaled to [0, M)."""
+    key = (h * M + i) * num_random + r
+    u = (splitmix64_output(seed, key + 1) >> 11) * (1.0 / (1 << 53))
+    return min(int(u * M), M - 1)
+
+
+def bigbird_cols(h: int, i: int, M: int, w: int, globals_: Sequence[int], num_random: int,
+                 seed: int, causal: bool = False) -> List[int]:
+    """BigBird's three kinds of connections ("Block Sparse Attention with
+    Log-Linear Complexity", section 2.2; parameters of the SparseFlashAttention
+    article's bigbird example): window |i - j| <= w, global blocks (full row and
+    full column) and num_random random columns drawn with replacement."""
+    if i in set(globals_):
+        cols = set(range(M))
+    else:
+        cols = {j for j in range(M) if abs(i - j) <= w}
+        cols.update(g for g in globals_ if 0 <= g < M)
+        cols.update(bigbird_random_col(seed, h, i, r, M, num_random) for r in range(num_random))
+    return sorted(j for j in cols if 0 <= j < M and (not causal or j <= i))
+
+
 def row_cols(desc, h: int, i: int) -> List[int]:
     """Columns of block row i of head h for a workloads.PatternDesc."""
     kind = desc.kind
@@ -103,6 +135,11 @@ def row_cols(desc, h: int, i: int) -> List[int]:
         return local_global_cols(i, desc.M, desc.local_radius, desc.anchors, desc.causal)
     if kind == 2:
         return bernoulli_cols(h, i, desc.M, desc.p, desc.seed, desc.causal)
+    if kind == 3:
+        return sliding_window_cols(i, desc.M, desc.local_radius, desc.dilation, desc.causal)
+    if kind == 4:
+        return bigbird_cols(h, i, desc.M, desc.local_radius, desc.anchors, desc.num_random,
+                            desc.seed, desc.causal)
     raise ValueError(f"unknown pattern kind {kind}")
 
 
@@ -110,7 +147,7 @@ def csr(desc) -> Tuple[np.ndarray, np.ndarray]:
     """Block-CSR over H*M rows (head-major): row_ptr int32 [H*M+1], col_idx int32 [nnz]."""
     M, H = desc.M, desc.H
     rows: List[List[int]] = []
-    if desc.kind == 2:
+    if desc.kind == 2 or (desc.kind == 4 and desc.num_random > 0):  # drawn per head
         for h in range(H):
             for i in range(M):
                 rows.append(row_cols(desc, h, i))

@@ -63,10 +63,17 @@ def _cases():
             out.append(PatternDesc(kind=2, M=M, H=3, p=0.3, seed=7, causal=causal))
             out.append(PatternDesc(kind=2, M=M, H=2, p=0.0, seed=1, causal=causal))
             out.append(PatternDesc(kind=2, M=M, H=2, p=1.0, seed=2 ** 64 - 1, causal=causal))
+            out.append(PatternDesc(kind=3, M=M, H=2, local_radius=min(8, M), dilation=2,
+                                   causal=causal))
+            out.append(PatternDesc(kind=3, M=M, H=1, local_radius=5, dilation=3, causal=causal))
+            out.append(PatternDesc(kind=4, M=M, H=3, local_radius=1, anchors=(0,), num_random=3,
+                                   seed=11, causal=causal))
+            out.append(PatternDesc(kind=4, M=M, H=2, local_radius=0, anchors=(M - 1, M // 2),
+                                   num_random=0, seed=5, causal=causal))
     return out
 
 
-@pytest.mark.parametrize("desc", _cases(), ids=lambda d: f"k{d.kind}M{d.M}H{d.H}c{int(d.causal)}r{d.local_radius}")
+@pytest.mark.parametrize("desc", _cases(), ids=lambda d: f"k{d.kind}M{d.M}H{d.H}c{int(d.causal)}r{d.local_radius}s{d.dilation}n{d.num_random}")
 def test_builder_matches_oracle_enumeration(desc):
     rp, ci = bsa.build_pattern_from(desc)
     orp, oci = patterns.csr(desc)
@@ -75,7 +82,7 @@ def test_builder_matches_oracle_enumeration(desc):
     assert bsa.validate_pattern(rp, ci, desc.H, desc.M, desc.causal) == bsa.OK
 
 
-@pytest.mark.parametrize("name", workloads.ORDER)
+@pytest.mark.parametrize("name", workloads.ORDER + workloads.EXTRA_ORDER)
 def test_builder_matches_oracle_on_workloads(name):
     d = workloads.WORKLOADS[name].pattern
     rp, ci = bsa.build_pattern_from(d)
@@ -86,7 +93,8 @@ def test_builder_matches_oracle_on_workloads(name):
 def test_builder_two_call_and_errors():
     lib = bsa.library()
     anc = (ctypes.c_int32 * 3)(0, 4, 7)
-    d = bsa._Desc(0, 8, 2, 1, 2, 3, ctypes.cast(anc, ctypes.POINTER(ctypes.c_int32)), 0.0, 0, 0)
+    d = bsa._Desc(0, 8, 2, 1, 2, 3, ctypes.cast(anc, ctypes.POINTER(ctypes.c_int32)), 0.0, 0, 0,
+                  1, 0)
     nnz = ctypes.c_int64(-1)
     assert lib.bsa_build_pattern(ctypes.byref(d), None, None, 0, ctypes.byref(nnz)) == bsa.OK
     assert nnz.value == 104
@@ -106,6 +114,14 @@ def test_builder_two_call_and_errors():
                                      ctypes.byref(nnz)) == bsa.ERR_INVALID_ARG, field
     dd = bsa._Desc.from_buffer_copy(d)
     dd.kind, dd.p = 2, 1.5
+    assert lib.bsa_build_pattern(ctypes.byref(dd), None, None, 0,
+                                 ctypes.byref(nnz)) == bsa.ERR_INVALID_ARG
+    dd = bsa._Desc.from_buffer_copy(d)
+    dd.kind, dd.dilation = 3, 0
+    assert lib.bsa_build_pattern(ctypes.byref(dd), None, None, 0,
+                                 ctypes.byref(nnz)) == bsa.ERR_INVALID_ARG
+    dd = bsa._Desc.from_buffer_copy(d)
+    dd.kind, dd.num_random = 4, -1
     assert lib.bsa_build_pattern(ctypes.byref(dd), None, None, 0,
                                  ctypes.byref(nnz)) == bsa.ERR_INVALID_ARG
     dd = bsa._Desc.from_buffer_copy(d)

@@ -76,7 +76,7 @@ def _sample_rows(w, rng, n_random):
     return np.array(sorted(rows), dtype=np.int64)
 
 
-@pytest.mark.parametrize("name", workloads.ORDER)
+@pytest.mark.parametrize("name", workloads.ORDER + workloads.EXTRA_ORDER)
 def test_workload_parity(name):
     w = workloads.WORKLOADS[name]
     q, k, v = workloads.make_qkv(w)

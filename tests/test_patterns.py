@@ -156,3 +156,48 @@ def test_csr_invariants(name):
 def test_causal_loglinear_first_row_is_diagonal_only():
     d = workloads.WORKLOADS["causal_loglinear_32k"].pattern
     assert patterns.loglinear_cols(0, d.M, d.log_kmax, d.anchors, 1, True) == [0]
+
+
+def test_sliding_window_matches_hand_enumeration():
+    # M = 10, window 4 blocks each side, every second block: rows written out
+    expect = {0: [0, 2, 4], 1: [1, 3, 5], 4: [0, 2, 4, 6, 8], 5: [1, 3, 5, 7, 9], 9: [5, 7, 9]}
+    for i, cols in expect.items():
+        assert patterns.sliding_window_cols(i, 10, 4, 2) == cols
+    # dilation 1 is the plain band; causal keeps j <= i
+    assert patterns.sliding_window_cols(3, 10, 2, 1) == [1, 2, 3, 4, 5]
+    assert patterns.sliding_window_cols(5, 10, 4, 2, causal=True) == [1, 3, 5]
+
+
+def test_bigbird_rows_are_window_globals_and_the_drawn_columns():
+    M, H, w, seed, R = 64, 3, 1, 11, 3
+    for h in range(H):
+        for i in range(M):
+            cols = patterns.bigbird_cols(h, i, M, w, (0,), R, seed)
+            if i == 0:
+                assert cols == list(range(M))              # a global row sees every block
+                continue
+            drawn = {patterns.bigbird_random_col(seed, h, i, r, M, R) for r in range(R)}
+            # the draw is output key+1 of the stream, key = (h*M + i)*R + r
+            key = (h * M + i) * R
+            u = (patterns.splitmix64_output(seed, key + 1) >> 11) / float(1 << 53)
+            assert patterns.bigbird_random_col(seed, h, i, 0, M, R) == int(u * M)
+            band = {j for j in range(i - w, i + w + 1) if 0 <= j < M}
+            assert set(cols) == band | {0} | drawn
+    # random columns differ between heads; with no random draws the heads repeat
+    rows = [tuple(patterns.bigbird_cols(h, 20, M, w, (0,), R, seed)) for h in range(H)]
+    assert len(set(rows)) > 1
+    assert patterns.bigbird_cols(1, 20, M, w, (0,), 0, seed) == patterns.bigbird_cols(0, 20, M, w, (0,), 0, seed)
+
+
+def test_bigbird_random_columns_spread_over_the_row():
+    M, R, seed = 64, 3, 11
+    hits = np.zeros(M)
+    for h in range(16):
+        for i in range(M):
+            for r in range(R):
+                hits[patterns.bigbird_random_col(seed, h, i, r, M, R)] += 1
+    expect = 16 * M * R / M
+    # chi-square over 64 cells, 63 degrees of freedom: far below the 0.1 % tail (~104)
+    chi2 = float(((hits - expect) ** 2 / expect).sum())
+    assert chi2 < 104.0
+

@@ -34,8 +34,11 @@ from typing import Optional, Tuple
 LOGLINEAR = 0
 LOCAL_GLOBAL = 1
 BERNOULLI = 2
+SLIDING_WINDOW = 3
+BIGBIRD = 4
 
-KIND_NAMES = {LOGLINEAR: "loglinear", LOCAL_GLOBAL: "local_global", BERNOULLI: "bernoulli"}
+KIND_NAMES = {LOGLINEAR: "loglinear", LOCAL_GLOBAL: "local_global", BERNOULLI: "bernoulli",
+              SLIDING_WINDOW: "sliding_window", BIGBIRD: "bigbird"}
 
 
 @dataclasses.dataclass(frozen=True)
@@ -51,6 +54,8 @@ class PatternDesc:
     p: float = 0.0              # BERNOULLI keep probability
     seed: int = 0               # BERNOULLI counter-based generator seed
     causal: bool = False        # keep only columns j <= i
+    dilation: int = 1           # SLIDING_WINDOW: keep j with (i - j) % dilation == 0
+    num_random: int = 0         # BIGBIRD: random columns drawn per block row
 
 
 @dataclasses.dataclass(frozen=True)
@@ -102,6 +107,30 @@ WORKLOADS = {
 
 # The same five workloads in the order they are usually listed.
 ORDER = ["tiny_loglinear", "loglinear_4k", "local_global_8k", "bernoulli_4k", "causal_loglinear_32k"]
+
+# The other pattern kinds of the pages, on shapes of the same scale (the
+# kernel is the same; only the block-CSR differs):
+#  - dilated sliding window: 512 tokens each side at block 64 (8 blocks),
+#    every second block (the SparseFlashAttention article's example);
+#  - BigBird: 3-block window, block 0 global, 3 random blocks per row, block 64
+#    (the same article's example; random blocks drawn per head);
+#  - log-linear with seven anchors instead of three ("Block Sparse Attention
+#    with Log-Linear Complexity", section 6.1).
+EXTRA = {
+    "sliding_window_8k": Workload(
+        "sliding_window_8k", 1, 16, 8192, 128, 64,
+        PatternDesc(kind=SLIDING_WINDOW, M=128, H=16, local_radius=8, dilation=2), seed=5),
+    "bigbird_4k": Workload(
+        "bigbird_4k", 2, 16, 4096, 64, 64,
+        PatternDesc(kind=BIGBIRD, M=64, H=16, local_radius=1, anchors=(0,), num_random=3, seed=11),
+        seed=6),
+    "loglinear7_4k": Workload(
+        "loglinear7_4k", 1, 16, 4096, 64, 32,
+        PatternDesc(kind=LOGLINEAR, M=128, H=16, local_radius=1, log_kmax=6,
+                    anchors=(0, 8, 32, 64, 96, 120, 127)), seed=7),
+}
+WORKLOADS.update(EXTRA)
+EXTRA_ORDER = list(EXTRA)
 
 
 def make_qkv(w: Workload, seed: Optional[int] = None):
