@@ -207,14 +207,31 @@ def cpu_oracle_sample(w, q, k, v, rp, ci, seconds: float, rng_seed: int = 0):
     return flops / elapsed / 1e12, threads, done_rows, elapsed
 
 
+def oracle_problem(w, q, k, v):
+    """The oracle's view of workload w: (workload, q, k, v, row_ptr, col_idx).
+    A top-k workload's pattern is the oracle's own selection, one CSR row per
+    (b, h, block row), with the batch folded into the heads."""
+    from oracle import patterns
+
+    if w.pattern.kind != workloads.TOPK:
+        rp, ci = patterns.csr(w.pattern)
+        return w, q, k, v, rp, ci
+    from oracle import topk as topk_oracle
+
+    rp, ci = topk_oracle.topk_pattern(q.float().numpy(), k.float().numpy(), w.block_size,
+                                      w.pattern.top_k, w.causal)
+    wf = workloads.Workload(w.name, 1, w.B * w.H, w.N, w.d, w.block_size, w.pattern, w.seed,
+                            causal=w.causal)
+    shape = (1, w.B * w.H, w.N, w.d)
+    return wf, q.reshape(shape), k.reshape(shape), v.reshape(shape), rp, ci
+
+
 def run_reference(args, w, rank, world):
     """fp64 CPU oracle on the host cores, each step a bounded sample of rows."""
     if rank != 0:
         return
-    from oracle import patterns
-
-    q, k, v = workloads.make_qkv(w)
-    rp, ci = patterns.csr(w.pattern)
+    w_in = w
+    w, q, k, v, rp, ci = oracle_problem(w, *workloads.make_qkv(w))
     step_seconds = 2.0
     for i in range(args.warmup):
         cpu_oracle_sample(w, q, k, v, rp, ci, 0.2, rng_seed=1000 + i)
@@ -231,8 +248,8 @@ def run_reference(args, w, rank, world):
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * statistics.mean(times), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d,
-                   "block_size": w.block_size},
+        "config": {"workload": w_in.name, "B": w_in.B, "H": w_in.H, "N": w_in.N, "d": w_in.d,
+                   "block_size": w_in.block_size},
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
                          "sample": f"{rows_done} random query rows of {w.name} over {args.steps} steps"},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -252,19 +269,35 @@ def run_ours(args, w, rank, world, local_rank):
 
     # Inputs: each rank its own replica (seed offset by rank).
     q_h, k_h, v_h = workloads.make_qkv(w, seed=replica_seed(w, rank))
-    rp_np, ci_np = bsa.build_pattern_from(w.pattern)
-    nnz = int(len(ci_np))
-    flops = useful_flops(w, nnz)
     q, k, v = q_h.to(dev), k_h.to(dev), v_h.to(dev)
-    rp = torch.from_numpy(rp_np).to(dev)
-    ci = torch.from_numpy(ci_np).to(dev)
     O = torch.empty_like(q)
     L = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=dev)
     flush = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
+    topk = w.pattern.kind == workloads.TOPK
+    if topk:
+        # The step chooses the pattern on the device from Q and K, then runs
+        # the forward on it with the batch folded into the heads.
+        fold = (1, w.B * w.H, w.N, w.d)
+        ws = torch.empty(bsa.library().bsa_topk_workspace_bytes(w.B * w.H, w.N, w.d, w.block_size) // 8,
+                         dtype=torch.float64, device=dev)
+        rp, ci = bsa.topk_pattern(q, k, w.block_size, w.pattern.top_k, w.causal, workspace=ws)
+        rp_np, ci_np = rp.cpu().numpy(), ci.cpu().numpy()
 
-    def step():
-        bsa.forward(q, k, v, rp, ci, w.block_size, w.scale, w.causal, out=O, lse=L)
+        def step():
+            rp_s, ci_s = bsa.topk_pattern(q, k, w.block_size, w.pattern.top_k, w.causal,
+                                          workspace=ws)
+            bsa.forward(q.view(fold), k.view(fold), v.view(fold), rp_s, ci_s, w.block_size,
+                        w.scale, w.causal, out=O.view(fold), lse=L.view(fold[:3]))
+    else:
+        rp_np, ci_np = bsa.build_pattern_from(w.pattern)
+        rp = torch.from_numpy(rp_np).to(dev)
+        ci = torch.from_numpy(ci_np).to(dev)
+
+        def step():
+            bsa.forward(q, k, v, rp, ci, w.block_size, w.scale, w.causal, out=O, lse=L)
+    nnz = int(len(ci_np))
+    flops = useful_flops(w, nnz)
 
     for _ in range(args.warmup):
         flush.fill_(1)
@@ -309,14 +342,28 @@ def run_ours(args, w, rank, world, local_rank):
     cip = torch.from_numpy(ci_np).pin_memory()
     Oh = torch.empty(q_h.shape, dtype=torch.bfloat16).pin_memory()
     Lh = torch.empty((w.B, w.H, w.N), dtype=torch.float32).pin_memory()
-    h2d = sum(t.numel() * t.element_size() for t in (qp, kp, vp, rpp, cip))
+    h2d = sum(t.numel() * t.element_size() for t in ((qp, kp, vp) if topk else (qp, kp, vp, rpp, cip)))
     d2h = Oh.numel() * Oh.element_size() + Lh.numel() * Lh.element_size()
     qd, kd, vd = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     rpd, cid = torch.empty_like(rp), torch.empty_like(ci)
     chunks = e2e_chunks(w)
     s_in, s_fw, s_out = (torch.cuda.Stream(dev) for _ in range(3))
 
+    def e2e_step_topk():
+        # host inputs in, pattern chosen on the device, forward, result out
+        with torch.cuda.stream(stream):
+            for dst, src in ((qd, qp), (kd, kp), (vd, vp)):
+                dst.copy_(src, non_blocking=True)
+            rp_s, ci_s = bsa.topk_pattern(qd, kd, w.block_size, w.pattern.top_k, w.causal,
+                                          workspace=ws)
+            bsa.forward(qd.view(fold), kd.view(fold), vd.view(fold), rp_s, ci_s, w.block_size,
+                        w.scale, w.causal, out=O.view(fold), lse=L.view(fold[:3]))
+            Oh.copy_(O, non_blocking=True)
+            Lh.copy_(L, non_blocking=True)
+
     def e2e_step():
+        if topk:
+            return e2e_step_topk()
         s_in.wait_stream(stream)
         with torch.cuda.stream(s_in):
             rpd.copy_(rpp, non_blocking=True)
@@ -387,10 +434,8 @@ def run_ours(args, w, rank, world, local_rank):
     # CPU baseline: the oracle, as it stands, on a bounded sample of rows.
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
-        from oracle import patterns
-
-        orp, oci = patterns.csr(w.pattern)
-        tf, threads, nrows, el = cpu_oracle_sample(w, q_h, k_h, v_h, orp, oci, args.cpu_seconds)
+        wo, qo, ko, vo, orp, oci = oracle_problem(w, q_h, k_h, v_h)
+        tf, threads, nrows, el = cpu_oracle_sample(wo, qo, ko, vo, orp, oci, args.cpu_seconds)
         cpu = {"value": tf, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
                "sample": f"{nrows} random query rows of {w.name} ({el:.1f} s, fp64)"}
 

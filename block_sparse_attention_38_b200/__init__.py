@@ -88,6 +88,13 @@ def library() -> ctypes.CDLL:
         lib.bsa_device_status.argtypes = [ctypes.POINTER(ctypes.c_uint32), ctypes.c_int]
         lib.bsa_version.restype = ctypes.c_int
         lib.bsa_version.argtypes = []
+        lib.bsa_topk_nnz.restype = ctypes.c_int64
+        lib.bsa_topk_nnz.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int]
+        lib.bsa_topk_workspace_bytes.restype = ctypes.c_size_t
+        lib.bsa_topk_workspace_bytes.argtypes = [ctypes.c_int] * 4
+        lib.bsa_topk_pattern.restype = ctypes.c_int
+        lib.bsa_topk_pattern.argtypes = [vp, vp] + [ctypes.c_int] * 6 + [vp, vp, vp,
+                                                                          ctypes.c_size_t, vp]
         _lib = lib
     return _lib
 
@@ -172,6 +179,50 @@ def forward(q, k, v, row_ptr, col_idx, block_size: int, scale: Optional[float] =
                              int(bool(causal)), out.data_ptr(), lse.data_ptr(), stream)
     _check(rc, "bsa_forward")
     return out, lse
+
+
+def topk_nnz(BH: int, M: int, top_k: int, causal: bool = False) -> int:
+    """Stored blocks of a top-k pattern over BH heads (bsa_topk_nnz)."""
+    n = int(library().bsa_topk_nnz(int(BH), int(M), int(top_k), int(bool(causal))))
+    if n < 0:
+        raise BsaError(ERR_INVALID_ARG, "bsa_topk_nnz")
+    return n
+
+
+def topk_pattern(q, k, block_size: int, top_k: int, causal: bool = False, workspace=None):
+    """Content-based top-k block selection on q's device (bsa_topk_pattern).
+
+    q, k: CUDA bf16 [B, H, N, d] contiguous.  Returns device int32 (row_ptr
+    [B*H*M+1], col_idx) with one CSR row per (b*H + h, block row): run
+    `forward` on q.view(1, B*H, N, d) etc. with it.  The fp64 workspace is a
+    caller-owned CUDA tensor (allocated here when not given).
+    """
+    import torch
+
+    lib = library()
+    if q.dim() != 4 or k.shape != q.shape:
+        raise ValueError("q, k must share one shape [B, H, N, d]")
+    for name, t in (("q", q), ("k", k)):
+        if not t.is_cuda or t.dtype != torch.bfloat16 or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous CUDA bf16 tensor")
+    B, H, N, d = (int(x) for x in q.shape)
+    BH, M = B * H, N // int(block_size)
+    nbytes = int(lib.bsa_topk_workspace_bytes(BH, N, d, int(block_size)))
+    if nbytes == 0:
+        raise BsaError(ERR_INVALID_ARG, "bsa_topk_workspace_bytes")
+    if workspace is None:
+        workspace = torch.empty(nbytes // 8, dtype=torch.float64, device=q.device)
+    nnz = topk_nnz(BH, M, top_k, causal)
+    row_ptr = torch.empty(BH * M + 1, dtype=torch.int32, device=q.device)
+    col_idx = torch.empty(max(nnz, 1), dtype=torch.int32, device=q.device)
+    with torch.cuda.device(q.device):
+        stream = torch.cuda.current_stream(q.device).cuda_stream
+        rc = lib.bsa_topk_pattern(q.data_ptr(), k.data_ptr(), BH, N, d, int(block_size),
+                                  int(top_k), int(bool(causal)), row_ptr.data_ptr(),
+                                  col_idx.data_ptr(), workspace.data_ptr(),
+                                  workspace.numel() * workspace.element_size(), stream)
+    _check(rc, "bsa_topk_pattern")
+    return row_ptr, col_idx[:nnz]
 
 
 def device_status(clear: bool = True) -> int:

@@ -1,0 +1,203 @@
+// bsa_topk.cu -- content-based top-k block selection on the device.
+//
+// The SparseFlashAttention article ("pattern generation", third kind) picks
+// the Top-K positions by the similarity of Q and K; here, at block level, row
+// i keeps its diagonal block and the top_k blocks j (j != i, j <= i when
+// causal) of highest s[i, j] = Qm[i] . Km[j], Qm and Km the block means of Q
+// and K.  The selection is an integer decision, so the arithmetic is pinned
+// to fp64 in a fixed order with every operation rounded on its own
+// (__dadd_rn / __dmul_rn: no fused multiply-add): tokens added in ascending
+// order, then products over c in ascending order.
+//
+//   means_kernel   one CTA per (bh, block), one thread per column c
+//   select_kernel  one CTA per (bh, block row): scores of the M candidate
+//                  blocks into shared memory, a bitonic sort on (score
+//                  descending, column ascending), then the chosen columns
+//                  written in ascending order at the row's fixed CSR offset
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+
+#include "bsa.h"
+
+namespace bsa {
+namespace topk {
+
+constexpr int kMaxM = 4096;
+constexpr int kMaxD = 256;
+constexpr int kSelectThreads = 256;
+
+__host__ __device__ inline int64_t row_length(int64_t i, int64_t M, int64_t top_k, int causal) {
+  const int64_t others = causal ? i : M - 1;
+  return 1 + (top_k < others ? top_k : others);
+}
+
+// Stored blocks of rows 0..i-1 of one (bh).
+__host__ __device__ inline int64_t row_offset(int64_t i, int64_t M, int64_t top_k, int causal) {
+  if (!causal) return i * (1 + (top_k < M - 1 ? top_k : M - 1));
+  // sum over i' < i of 1 + min(top_k, i')
+  const int64_t m = i < top_k ? i : top_k;
+  const int64_t tail = i > top_k ? (i - top_k) * top_k : 0;
+  return i + m * (m - 1) / 2 + tail;
+}
+
+__global__ void means_kernel(const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* __restrict__ K,
+                             int d, int bs, double* __restrict__ qm, double* __restrict__ km) {
+  const long long blk = blockIdx.x;  // bh * M + i: tokens blk*bs .. blk*bs + bs - 1
+  const int c = threadIdx.x;
+  if (c >= d) return;
+  const long long base = blk * bs * d + c;
+  double sq = 0.0, sk = 0.0;
+  for (int t = 0; t < bs; ++t) {
+    sq = __dadd_rn(sq, static_cast<double>(__bfloat162float(Q[base + static_cast<long long>(t) * d])));
+    sk = __dadd_rn(sk, static_cast<double>(__bfloat162float(K[base + static_cast<long long>(t) * d])));
+  }
+  const double inv = 1.0 / bs;  // exact: bs is a power of two in practice, and the oracle divides
+  qm[blk * d + c] = bs == (bs & -bs) ? __dmul_rn(sq, inv) : __ddiv_rn(sq, static_cast<double>(bs));
+  km[blk * d + c] = bs == (bs & -bs) ? __dmul_rn(sk, inv) : __ddiv_rn(sk, static_cast<double>(bs));
+}
+
+// a before b: higher score, then smaller column.
+__device__ inline bool before(double sa, int ja, double sb, int jb) {
+  return sa > sb || (sa == sb && ja < jb);
+}
+
+__global__ void __launch_bounds__(kSelectThreads)
+    select_kernel(const double* __restrict__ qm, const double* __restrict__ km, int M, int Mp,
+                  int d, int top_k, int causal, int32_t* __restrict__ row_ptr,
+                  int32_t* __restrict__ col_idx, long long num_rows) {
+  extern __shared__ unsigned char smem_raw[];
+  double* score = reinterpret_cast<double*>(smem_raw);          // [Mp]
+  double* qrow = score + Mp;                                   // [d]
+  int* idx = reinterpret_cast<int*>(qrow + kMaxD);             // [Mp]
+  unsigned char* chosen = reinterpret_cast<unsigned char*>(idx + Mp);  // [Mp]
+  __shared__ int warp_sum[kSelectThreads / 32];
+
+  const long long r = blockIdx.x;  // bh * M + i
+  const long long bh = r / M;
+  const int i = static_cast<int>(r - bh * M);
+  const int tid = threadIdx.x;
+  for (int c = tid; c < d; c += kSelectThreads) qrow[c] = qm[r * d + c];
+  __syncthreads();
+
+  const double* kbase = km + bh * static_cast<long long>(M) * d;
+  for (int j = tid; j < Mp; j += kSelectThreads) {
+    double s = -INFINITY;  // not a candidate: sorts after every finite score
+    if (j < M && j != i && (!causal || j <= i)) {
+      s = 0.0;
+      const double* kr = kbase + static_cast<long long>(j) * d;
+      for (int c = 0; c < d; ++c) s = __dadd_rn(s, __dmul_rn(qrow[c], kr[c]));
+    }
+    score[j] = s;
+    idx[j] = j;
+    chosen[j] = 0;
+  }
+  __syncthreads();
+
+  // Bitonic sort of (score, column) over Mp (a power of two) entries.
+  for (int size = 2; size <= Mp; size <<= 1) {
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      for (int p = tid; p < Mp / 2; p += kSelectThreads) {
+        const int lo = 2 * p - (p & (stride - 1));  // first element of the pair
+        const int hi = lo + stride;
+        const bool up = (lo & size) == 0;           // this run sorts in "before" order
+        const bool swap = up ? before(score[hi], idx[hi], score[lo], idx[lo])
+                             : before(score[lo], idx[lo], score[hi], idx[hi]);
+        if (swap) {
+          const double ts = score[lo];
+          score[lo] = score[hi];
+          score[hi] = ts;
+          const int ti = idx[lo];
+          idx[lo] = idx[hi];
+          idx[hi] = ti;
+        }
+      }
+      __syncthreads();
+    }
+  }
+
+  const int keep = static_cast<int>(row_length(i, M, top_k, causal)) - 1;  // chosen besides i
+  for (int p = tid; p < keep; p += kSelectThreads) chosen[idx[p]] = 1;
+  if (tid == 0) chosen[i] = 1;
+  __syncthreads();
+
+  // Chosen columns in ascending order: each thread owns a contiguous range.
+  const int per = (M + kSelectThreads - 1) / kSelectThreads;
+  const int j0 = tid * per, j1 = min(M, j0 + per);
+  int cnt = 0;
+  for (int j = j0; j < j1; ++j) cnt += chosen[j];
+  const int lane = tid & 31, warp = tid >> 5;
+  int incl = cnt;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += v;
+  }
+  if (lane == 31) warp_sum[warp] = incl;
+  __syncthreads();
+  int base = 0;
+  for (int w = 0; w < warp; ++w) base += warp_sum[w];
+  const long long row_start = bh * row_offset(M, M, top_k, causal) + row_offset(i, M, top_k, causal);
+  int pos = base + incl - cnt;
+  for (int j = j0; j < j1; ++j)
+    if (chosen[j]) col_idx[row_start + pos++] = j;
+  if (tid == 0) {
+    row_ptr[r] = static_cast<int32_t>(row_start);
+    if (r == num_rows - 1)
+      row_ptr[num_rows] = static_cast<int32_t>(row_start + row_length(i, M, top_k, causal));
+  }
+}
+
+}  // namespace topk
+}  // namespace bsa
+
+extern "C" int64_t bsa_topk_nnz(int BH, int M, int top_k, int causal) {
+  if (BH < 1 || M < 1 || top_k < 0 || (causal != 0 && causal != 1)) return -1;
+  return static_cast<int64_t>(BH) * bsa::topk::row_offset(M, M, top_k, causal);
+}
+
+extern "C" size_t bsa_topk_workspace_bytes(int BH, int N, int d, int block_size) {
+  if (BH < 1 || N < 1 || d < 1 || block_size < 1 || N % block_size != 0) return 0;
+  return 2ull * static_cast<size_t>(BH) * static_cast<size_t>(N / block_size) *
+         static_cast<size_t>(d) * sizeof(double);
+}
+
+extern "C" int bsa_topk_pattern(const void* Q, const void* K, int BH, int N, int d,
+                                int block_size, int top_k, int causal, int32_t* row_ptr,
+                                int32_t* col_idx, void* workspace, size_t workspace_bytes,
+                                void* stream) {
+  using namespace bsa::topk;
+  if (!Q || !K || !row_ptr || !col_idx || !workspace) return BSA_ERR_INVALID_ARG;
+  if (BH < 1 || N < 1 || d < 1 || block_size < 1 || top_k < 0) return BSA_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return BSA_ERR_INVALID_ARG;
+  if (N % block_size != 0) return BSA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 7u) != 0) return BSA_ERR_INVALID_ARG;
+  const int M = N / block_size;
+  if (d > kMaxD || M > kMaxM) return BSA_ERR_UNSUPPORTED;
+  const int64_t nnz = bsa_topk_nnz(BH, M, top_k, causal);
+  if (static_cast<int64_t>(BH) * M + 1 > INT32_MAX || nnz > INT32_MAX) return BSA_ERR_UNSUPPORTED;
+  if (workspace_bytes < bsa_topk_workspace_bytes(BH, N, d, block_size)) return BSA_ERR_BUFFER_TOO_SMALL;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  double* qm = static_cast<double*>(workspace);
+  double* km = qm + static_cast<size_t>(BH) * M * d;
+  const long long blocks = static_cast<long long>(BH) * M;
+  means_kernel<<<static_cast<unsigned>(blocks), d, 0, s>>>(
+      static_cast<const __nv_bfloat16*>(Q), static_cast<const __nv_bfloat16*>(K), d, block_size,
+      qm, km);
+  if (cudaGetLastError() != cudaSuccess) return BSA_ERR_CUDA;
+  int Mp = 1;
+  while (Mp < M) Mp <<= 1;
+  if (Mp < 2) Mp = 2;
+  const size_t smem = static_cast<size_t>(Mp) * sizeof(double) + kMaxD * sizeof(double) +
+                      static_cast<size_t>(Mp) * sizeof(int) + static_cast<size_t>(Mp);
+  if (smem > 48 * 1024 &&
+      cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(smem)) != cudaSuccess)
+    return BSA_ERR_CUDA;
+  select_kernel<<<static_cast<unsigned>(blocks), kSelectThreads, smem, s>>>(
+      qm, km, M, Mp, d, top_k, causal, row_ptr, col_idx, blocks);
+  if (cudaGetLastError() != cudaSuccess) return BSA_ERR_CUDA;
+  return BSA_OK;
+}

@@ -158,6 +158,49 @@ int bsa_forward(const void* Q, const void* K, const void* V,
 #define BSA_STATUS_BAD_ROW_PTR 0x4u  /* row_ptr[i+1] < row_ptr[i] was seen; the row was treated as empty */
 
 /*
+ * Content-based top-k block selection (a pattern computed from Q and K on the
+ * device).  The SparseFlashAttention article ("pattern generation", third
+ * kind) chooses the Top-K positions by the similarity of Q and K; the RTX
+ * 4090 article uses "dynamic sparsity, topk = 20%".  At block level:
+ *   Qm[i, c] = (sum over the bs tokens t of block i of Q[t, c]) / bs, Km alike;
+ *   s[i, j]  = sum over c of Qm[i, c] * Km[j, c];
+ *   row i keeps its diagonal block and the top_k highest-scoring other
+ *   allowed blocks (j != i; j <= i when causal), ties to the smaller j.
+ * All arithmetic is fp64 in a fixed order (tokens, then c, ascending; each
+ * product rounded on its own, no fused multiply-add), so that the selection
+ * is reproducible.  One CSR row per (b*H + h, i): run the forward on the
+ * result with the batch folded into the heads, [1, B*H, N, d].
+ *
+ * Row i holds 1 + min(top_k, i if causal else M - 1) columns, ascending, so
+ * row_ptr is fixed by (BH, M, top_k, causal); bsa_topk_nnz gives the total.
+ */
+
+/* Total stored blocks of a top-k pattern; -1 for BH < 1, M < 1 or top_k < 0. */
+int64_t bsa_topk_nnz(int BH, int M, int top_k, int causal);
+
+/* Device workspace bytes bsa_topk_pattern needs (the fp64 block means of Q
+ * and K): 2 * BH * (N / block_size) * d * 8; 0 for invalid sizes. */
+size_t bsa_topk_workspace_bytes(int BH, int N, int d, int block_size);
+
+/*
+ * bsa_topk_pattern -- the selection above, enqueued on `stream`.
+ *
+ * Q, K: device bf16 [BH, N, d] contiguous (BH = B*H).  row_ptr: device int32
+ * [BH*M+1]; col_idx: device int32 [bsa_topk_nnz(...)]; workspace: caller-owned
+ * device memory of at least bsa_topk_workspace_bytes(...) bytes, 8-byte
+ * aligned, which the call overwrites (it need not be zeroed).  Nothing is
+ * allocated and nothing synchronised.
+ * Supported: 1 <= d <= 256, block_size >= 1, N % block_size == 0,
+ * 1 <= M <= 4096, top_k >= 0, causal 0/1, BH >= 1.  Else
+ * BSA_ERR_INVALID_ARG / BSA_ERR_UNSUPPORTED with nothing launched;
+ * BSA_ERR_BUFFER_TOO_SMALL for a short workspace; BSA_ERR_CUDA if a launch
+ * fails.
+ */
+int bsa_topk_pattern(const void* Q, const void* K, int BH, int N, int d, int block_size,
+                     int top_k, int causal, int32_t* row_ptr, int32_t* col_idx,
+                     void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * bsa_device_status -- read (and with clear != 0, reset) the status word of
  * the current device.  Synchronises the device.  Returns BSA_OK or
  * BSA_ERR_CUDA; *status receives an OR of BSA_STATUS_* bits accumulated by

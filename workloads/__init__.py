@@ -36,9 +36,10 @@ LOCAL_GLOBAL = 1
 BERNOULLI = 2
 SLIDING_WINDOW = 3
 BIGBIRD = 4
+TOPK = 5  # chosen on the device from Q and K (not a host-builder kind)
 
 KIND_NAMES = {LOGLINEAR: "loglinear", LOCAL_GLOBAL: "local_global", BERNOULLI: "bernoulli",
-              SLIDING_WINDOW: "sliding_window", BIGBIRD: "bigbird"}
+              SLIDING_WINDOW: "sliding_window", BIGBIRD: "bigbird", TOPK: "topk"}
 
 
 @dataclasses.dataclass(frozen=True)
@@ -56,6 +57,7 @@ class PatternDesc:
     causal: bool = False        # keep only columns j <= i
     dilation: int = 1           # SLIDING_WINDOW: keep j with (i - j) % dilation == 0
     num_random: int = 0         # BIGBIRD: random columns drawn per block row
+    top_k: int = 0              # TOPK: blocks kept per row besides the diagonal
 
 
 @dataclasses.dataclass(frozen=True)
@@ -131,6 +133,16 @@ EXTRA = {
 }
 WORKLOADS.update(EXTRA)
 EXTRA_ORDER = list(EXTRA)
+
+# Content-based selection: each block row of each (b, h) keeps its diagonal
+# and the top_k blocks of highest mean-Q . mean-K score, chosen on the device
+# (20 % of the row, the RTX 4090 article's "topk = 20%").
+TOPK_WORKLOADS = {
+    "topk_4k": Workload(
+        "topk_4k", 1, 16, 4096, 64, 32,
+        PatternDesc(kind=TOPK, M=128, H=16, top_k=25), seed=8),
+}
+WORKLOADS.update(TOPK_WORKLOADS)
 
 
 def make_qkv(w: Workload, seed: Optional[int] = None):
