@@ -110,13 +110,16 @@ def compulsory_bytes(w) -> float:
     return 4.0 * w.B * w.H * w.N * w.d * 2 + 4.0 * w.B * w.H * w.N
 
 
+# The files the forward kernel is compiled from (bsa_forward.cu and what it includes).
+FORWARD_SOURCES = ("bsa_common.cuh", "bsa_forward.cu", "bsa_fwd_rows.cuh", "sm100_ptx.cuh")
+
+
 def kernel_hash() -> str:
-    """sha256 prefix over every kernel source file (sorted by name)."""
+    """sha256 prefix over the forward kernel's source files (sorted by name)."""
     h = hashlib.sha256()
-    for name in sorted(os.listdir(KERNEL_DIR)):
-        if name.endswith((".cu", ".cuh")):
-            with open(os.path.join(KERNEL_DIR, name), "rb") as f:
-                h.update(name.encode() + b"\0" + f.read())
+    for name in sorted(FORWARD_SOURCES):
+        with open(os.path.join(KERNEL_DIR, name), "rb") as f:
+            h.update(name.encode() + b"\0" + f.read())
     return h.hexdigest()[:16]
 
 
@@ -284,18 +287,24 @@ def run_ours(args, w, rank, world, local_rank):
         rp, ci = bsa.topk_pattern(q, k, w.block_size, w.pattern.top_k, w.causal, workspace=ws)
         rp_np, ci_np = rp.cpu().numpy(), ci.cpu().numpy()
 
-        def step():
+        def step(mid=None):
             rp_s, ci_s = bsa.topk_pattern(q, k, w.block_size, w.pattern.top_k, w.causal,
                                           workspace=ws)
+            if mid is not None:
+                mid.record(stream)
             bsa.forward(q.view(fold), k.view(fold), v.view(fold), rp_s, ci_s, w.block_size,
                         w.scale, w.causal, out=O.view(fold), lse=L.view(fold[:3]))
+        launches_per_step = 3  # block means, selection, forward
     else:
         rp_np, ci_np = bsa.build_pattern_from(w.pattern)
         rp = torch.from_numpy(rp_np).to(dev)
         ci = torch.from_numpy(ci_np).to(dev)
 
-        def step():
+        def step(mid=None):
+            if mid is not None:
+                mid.record(stream)
             bsa.forward(q, k, v, rp, ci, w.block_size, w.scale, w.causal, out=O, lse=L)
+        launches_per_step = 1
     nnz = int(len(ci_np))
     flops = useful_flops(w, nnz)
 
@@ -311,6 +320,7 @@ def run_ours(args, w, rank, world, local_rank):
     if rank == 0:
         clocks.start()
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    mids = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     if world > 1:
         dist.barrier()
@@ -318,7 +328,7 @@ def run_ours(args, w, rank, world, local_rank):
     for i in range(args.steps):
         flush.fill_(i & 0xFF)
         starts[i].record(stream)
-        step()
+        step(mids[i])
         ends[i].record(stream)
     torch.cuda.synchronize()
     if world > 1:
@@ -326,6 +336,8 @@ def run_ours(args, w, rank, world, local_rank):
     clock_info = clocks.stop() if rank == 0 else None
     per_step = [s.elapsed_time(e) for s, e in zip(starts, ends)]
     total_ms = float(sum(per_step))
+    # the forward kernel alone (for a top-k step, after the selection kernels)
+    fwd_ms_total = float(sum(m.elapsed_time(e) for m, e in zip(mids, ends)))
     status = bsa.device_status(clear=True)
     if status:
         raise RuntimeError(f"kernel reported device status {status:#x}")
@@ -407,11 +419,13 @@ def run_ours(args, w, rank, world, local_rank):
     if not torch.equal(Oh, ref_o):
         raise RuntimeError("end-to-end result differs from the device result")
 
-    total_ms, e2e_ms = max_over_ranks([total_ms, e2e_ms], world, device=dev)
+    total_ms, e2e_ms, fwd_ms_total = max_over_ranks([total_ms, e2e_ms, fwd_ms_total], world,
+                                                    device=dev)
     if rank != 0:
         return
 
     ms = total_ms / args.steps
+    fwd_ms = fwd_ms_total / args.steps
     value = whole_job_tflops(flops, world, ms)
     e2e_value = whole_job_tflops(flops, world, e2e_ms)
     peaks, peak_src = load_peaks()
@@ -420,16 +434,18 @@ def run_ours(args, w, rank, world, local_rank):
     t_tc = flops / (peak_tc * 1e12)
     t_hbm = compulsory_bytes(w) / (peak_hbm * 1e9)
     if t_tc >= t_hbm:
-        roof = {"bound": "tensor", "achieved": flops / (ms * 1e-3) / 1e12, "peak": peak_tc,
+        roof = {"bound": "tensor", "achieved": flops / (fwd_ms * 1e-3) / 1e12, "peak": peak_tc,
                 "unit": "TFLOP/s"}
     else:
-        roof = {"bound": "hbm", "achieved": compulsory_bytes(w) / (ms * 1e-3) / 1e9,
+        roof = {"bound": "hbm", "achieved": compulsory_bytes(w) / (fwd_ms * 1e-3) / 1e9,
                 "peak": peak_hbm, "unit": "GB/s"}
     roof["frac"] = roof["achieved"] / roof["peak"]
     tr = NCU_TRAFFIC.get(w.name)
     roof["traffic"] = tr[0] if tr and tr[1] == kernel_hash() else None
     roof["peak_source"] = f"{peak_src} (MEASURED_PEAKS.json burst)" if peak_src == "measured" else "fallback"
-    roof["roofline_frac_max_of_tc_hbm"] = max(t_tc, t_hbm) / (ms * 1e-3)
+    roof["roofline_frac_max_of_tc_hbm"] = max(t_tc, t_hbm) / (fwd_ms * 1e-3)
+    roof["kernel"] = "bsa::rows::fwd_kernel"
+    roof["kernel_ms"] = fwd_ms
 
     # CPU baseline: the oracle, as it stands, on a bounded sample of rows.
     cpu = None
@@ -452,10 +468,14 @@ def run_ours(args, w, rank, world, local_rank):
         "cpu_baseline": cpu,
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": int(h2d),
                 "d2h_bytes_per_step": int(d2h), "ms_per_step": e2e_ms},
-        "gpu_launches": args.steps,
+        "gpu_launches": args.steps * launches_per_step,
         "clocks": clock_info,
         "min_ms": min(per_step), "median_ms": statistics.median(per_step),
     }
+    if topk:
+        # the selection (block means + top-k select kernels) ahead of the forward
+        line["config"]["top_k"] = w.pattern.top_k
+        line["selection_ms"] = ms - fwd_ms
     print(json.dumps(line), flush=True)
 
 

@@ -9,7 +9,10 @@
 // (__dadd_rn / __dmul_rn: no fused multiply-add): tokens added in ascending
 // order, then products over c in ascending order.
 //
-//   means_kernel   one CTA per (bh, block), one thread per column c
+//   means_kernel   one CTA per (bh, block), one thread per column c; the K
+//                  means are stored transposed, [bh][c][block], so that the
+//                  threads of the selection (one per candidate block) read
+//                  consecutive addresses for each c
 //   select_kernel  one CTA per (bh, block row): scores of the M candidate
 //                  blocks into shared memory, a bitonic sort on (score
 //                  descending, column ascending), then the chosen columns
@@ -43,9 +46,13 @@ __host__ __device__ inline int64_t row_offset(int64_t i, int64_t M, int64_t top_
   return i + m * (m - 1) / 2 + tail;
 }
 
+// qm: [BH, M, d];  kmT: [BH, d, M].
 __global__ void means_kernel(const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* __restrict__ K,
-                             int d, int bs, double* __restrict__ qm, double* __restrict__ km) {
+                             int M, int d, int bs, double* __restrict__ qm,
+                             double* __restrict__ kmT) {
   const long long blk = blockIdx.x;  // bh * M + i: tokens blk*bs .. blk*bs + bs - 1
+  const long long bh = blk / M;
+  const int i = static_cast<int>(blk - bh * M);
   const int c = threadIdx.x;
   if (c >= d) return;
   const long long base = blk * bs * d + c;
@@ -56,7 +63,7 @@ __global__ void means_kernel(const __nv_bfloat16* __restrict__ Q, const __nv_bfl
   }
   const double inv = 1.0 / bs;  // exact: bs is a power of two in practice, and the oracle divides
   qm[blk * d + c] = bs == (bs & -bs) ? __dmul_rn(sq, inv) : __ddiv_rn(sq, static_cast<double>(bs));
-  km[blk * d + c] = bs == (bs & -bs) ? __dmul_rn(sk, inv) : __ddiv_rn(sk, static_cast<double>(bs));
+  kmT[(bh * d + c) * M + i] = bs == (bs & -bs) ? __dmul_rn(sk, inv) : __ddiv_rn(sk, static_cast<double>(bs));
 }
 
 // a before b: higher score, then smaller column.
@@ -65,7 +72,7 @@ __device__ inline bool before(double sa, int ja, double sb, int jb) {
 }
 
 __global__ void __launch_bounds__(kSelectThreads)
-    select_kernel(const double* __restrict__ qm, const double* __restrict__ km, int M, int Mp,
+    select_kernel(const double* __restrict__ qm, const double* __restrict__ kmT, int M, int Mp,
                   int d, int top_k, int causal, int32_t* __restrict__ row_ptr,
                   int32_t* __restrict__ col_idx, long long num_rows) {
   extern __shared__ unsigned char smem_raw[];
@@ -82,13 +89,13 @@ __global__ void __launch_bounds__(kSelectThreads)
   for (int c = tid; c < d; c += kSelectThreads) qrow[c] = qm[r * d + c];
   __syncthreads();
 
-  const double* kbase = km + bh * static_cast<long long>(M) * d;
+  const double* kbase = kmT + bh * static_cast<long long>(M) * d;
   for (int j = tid; j < Mp; j += kSelectThreads) {
     double s = -INFINITY;  // not a candidate: sorts after every finite score
     if (j < M && j != i && (!causal || j <= i)) {
       s = 0.0;
-      const double* kr = kbase + static_cast<long long>(j) * d;
-      for (int c = 0; c < d; ++c) s = __dadd_rn(s, __dmul_rn(qrow[c], kr[c]));
+      const double* kc = kbase + j;  // Km[j, c] at kc[c * M]
+      for (int c = 0; c < d; ++c) s = __dadd_rn(s, __dmul_rn(qrow[c], kc[static_cast<long long>(c) * M]));
     }
     score[j] = s;
     idx[j] = j;
@@ -181,11 +188,11 @@ extern "C" int bsa_topk_pattern(const void* Q, const void* K, int BH, int N, int
   if (workspace_bytes < bsa_topk_workspace_bytes(BH, N, d, block_size)) return BSA_ERR_BUFFER_TOO_SMALL;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   double* qm = static_cast<double*>(workspace);
-  double* km = qm + static_cast<size_t>(BH) * M * d;
+  double* kmT = qm + static_cast<size_t>(BH) * M * d;
   const long long blocks = static_cast<long long>(BH) * M;
   means_kernel<<<static_cast<unsigned>(blocks), d, 0, s>>>(
-      static_cast<const __nv_bfloat16*>(Q), static_cast<const __nv_bfloat16*>(K), d, block_size,
-      qm, km);
+      static_cast<const __nv_bfloat16*>(Q), static_cast<const __nv_bfloat16*>(K), M, d, block_size,
+      qm, kmT);
   if (cudaGetLastError() != cudaSuccess) return BSA_ERR_CUDA;
   int Mp = 1;
   while (Mp < M) Mp <<= 1;
@@ -197,7 +204,7 @@ extern "C" int bsa_topk_pattern(const void* Q, const void* K, int BH, int N, int
                            static_cast<int>(smem)) != cudaSuccess)
     return BSA_ERR_CUDA;
   select_kernel<<<static_cast<unsigned>(blocks), kSelectThreads, smem, s>>>(
-      qm, km, M, Mp, d, top_k, causal, row_ptr, col_idx, blocks);
+      qm, kmT, M, Mp, d, top_k, causal, row_ptr, col_idx, blocks);
   if (cudaGetLastError() != cudaSuccess) return BSA_ERR_CUDA;
   return BSA_OK;
 }
