@@ -95,6 +95,8 @@ def library() -> ctypes.CDLL:
         lib.bsa_topk_pattern.restype = ctypes.c_int
         lib.bsa_topk_pattern.argtypes = [vp, vp] + [ctypes.c_int] * 6 + [vp, vp, vp,
                                                                           ctypes.c_size_t, vp]
+        lib.bsa_topk_pattern_static.restype = ctypes.c_int
+        lib.bsa_topk_pattern_static.argtypes = [vp, vp] + [ctypes.c_int] * 6 + [vp, vp, vp]
         _lib = lib
     return _lib
 
@@ -222,6 +224,46 @@ def topk_pattern(q, k, block_size: int, top_k: int, causal: bool = False, worksp
                                   col_idx.data_ptr(), workspace.data_ptr(),
                                   workspace.numel() * workspace.element_size(), stream)
     _check(rc, "bsa_topk_pattern")
+    return row_ptr, col_idx[:nnz]
+
+
+TOPK_STATIC_SCRATCH_BYTES = 4 * 1024 * 1024
+
+
+def topk_pattern_static(q, k, block_size: int, top_k: int, causal: bool, row_ptr, col_idx):
+    """bsa_topk_pattern_static: the top-k selection with the library's own
+    static scratch, writing into the caller's device int32 row_ptr
+    [B*H*M+1] and col_idx [topk_nnz(...)].  Allocates nothing.
+
+    Requests needing more than TOPK_STATIC_SCRATCH_BYTES of workspace raise
+    BsaError(ERR_BUFFER_TOO_SMALL); calls overlapping in time on one device race.
+    """
+    import torch
+
+    lib = library()
+    if q.dim() != 4 or k.shape != q.shape:
+        raise ValueError("q, k must share one shape [B, H, N, d]")
+    for name, t in (("q", q), ("k", k)):
+        if not t.is_cuda or t.dtype != torch.bfloat16 or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous CUDA bf16 tensor")
+    B, H, N, d = (int(x) for x in q.shape)
+    BH, M = B * H, N // int(block_size)
+    nnz = topk_nnz(BH, M, top_k, causal)
+    for name, t, n in (("row_ptr", row_ptr, BH * M + 1), ("col_idx", col_idx, nnz)):
+        if (not t.is_cuda or t.device != q.device or t.dtype != torch.int32
+                or not t.is_contiguous() or t.numel() < n):
+            raise ValueError(f"{name} must be a contiguous int32 tensor on q's device "
+                             f"with at least {n} elements")
+    need = int(lib.bsa_topk_workspace_bytes(BH, N, d, int(block_size)))
+    with torch.cuda.device(q.device):
+        stream = torch.cuda.current_stream(q.device).cuda_stream
+        rc = lib.bsa_topk_pattern_static(q.data_ptr(), k.data_ptr(), BH, N, d, int(block_size),
+                                         int(top_k), int(bool(causal)), row_ptr.data_ptr(),
+                                         col_idx.data_ptr(), stream)
+    if rc == ERR_BUFFER_TOO_SMALL:
+        raise BsaError(rc, f"bsa_topk_pattern_static (needs {need} bytes of scratch, the "
+                           f"static scratch holds {TOPK_STATIC_SCRATCH_BYTES})")
+    _check(rc, "bsa_topk_pattern_static")
     return row_ptr, col_idx[:nnz]
 
 

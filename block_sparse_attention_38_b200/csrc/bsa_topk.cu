@@ -20,8 +20,10 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cmath>
 #include <cstdint>
+#include <mutex>
 
 #include "bsa.h"
 
@@ -207,4 +209,61 @@ extern "C" int bsa_topk_pattern(const void* Q, const void* K, int BH, int N, int
       qm, kmT, M, Mp, d, top_k, causal, row_ptr, col_idx, blocks);
   if (cudaGetLastError() != cudaSuccess) return BSA_ERR_CUDA;
   return BSA_OK;
+}
+
+// ---------------------------------------------------------------------------
+// bsa_topk_pattern_static: the same selection with its fp64 workspace in a
+// fixed scratch area of this library instead of caller memory.  Every device
+// gets its own copy of the array when the library's module loads there; its
+// address is looked up once per device, on the first call.  No element of the
+// scratch needs to start at zero: the means kernel writes every element the
+// selection then reads, within the same call.  Two calls that overlap in time
+// on one device share the area and race.
+namespace bsa {
+namespace topk {
+
+constexpr size_t kStaticScratchBytes = BSA_TOPK_STATIC_SCRATCH_BYTES;
+static __device__ __align__(256) double g_static_scratch[kStaticScratchBytes / sizeof(double)];
+
+constexpr int kMaxDevices = 64;
+std::atomic<void*> g_static_addr[kMaxDevices];
+std::mutex g_static_mu;
+
+// Address of this device's scratch, or nullptr if the lookup failed.
+void* static_scratch(int dev) {
+  void* p = g_static_addr[dev].load(std::memory_order_acquire);
+  if (p) return p;
+  std::lock_guard<std::mutex> lock(g_static_mu);
+  p = g_static_addr[dev].load(std::memory_order_relaxed);
+  if (!p) {
+    if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess) return nullptr;
+    g_static_addr[dev].store(p, std::memory_order_release);
+  }
+  return p;
+}
+
+}  // namespace topk
+}  // namespace bsa
+
+extern "C" int bsa_topk_pattern_static(const void* Q, const void* K, int BH, int N, int d,
+                                       int block_size, int top_k, int causal, int32_t* row_ptr,
+                                       int32_t* col_idx, void* stream) {
+  using namespace bsa::topk;
+  // The argument checks of bsa_topk_pattern, then the scratch limit: all
+  // before any CUDA call.
+  if (!Q || !K || !row_ptr || !col_idx) return BSA_ERR_INVALID_ARG;
+  if (BH < 1 || N < 1 || d < 1 || block_size < 1 || top_k < 0) return BSA_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return BSA_ERR_INVALID_ARG;
+  if (N % block_size != 0) return BSA_ERR_INVALID_ARG;
+  const int M = N / block_size;
+  if (d > kMaxD || M > kMaxM) return BSA_ERR_UNSUPPORTED;
+  const size_t need = bsa_topk_workspace_bytes(BH, N, d, block_size);
+  if (need > kStaticScratchBytes) return BSA_ERR_BUFFER_TOO_SMALL;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return BSA_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return BSA_ERR_UNSUPPORTED;
+  void* scratch = static_scratch(dev);
+  if (!scratch) return BSA_ERR_CUDA;
+  return bsa_topk_pattern(Q, K, BH, N, d, block_size, top_k, causal, row_ptr, col_idx, scratch,
+                          kStaticScratchBytes, stream);
 }

@@ -201,6 +201,39 @@ int bsa_topk_pattern(const void* Q, const void* K, int BH, int N, int d, int blo
                      void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * bsa_topk_pattern_static -- bsa_topk_pattern without a caller workspace and
+ * without any allocation.  The pages have no counterpart: this is an
+ * interface of this library only, for callers that must not allocate device
+ * memory around the selection.
+ *
+ * The fp64 block means live in a scratch array of the library itself (a
+ * file-scope __device__ array, 256-byte aligned, one copy per device) of
+ * BSA_TOPK_STATIC_SCRATCH_BYTES.  Its address is looked up with
+ * cudaGetSymbolAddress on the first call on each device (the current device
+ * at the call), so make that first call before any stream capture on that
+ * device.  The call makes no cudaMalloc, cudaFree or other allocating call.
+ *
+ * Arguments, layouts, results and the other errors are those of
+ * bsa_topk_pattern (same kernels, same bits).  A request whose workspace,
+ * bsa_topk_workspace_bytes(BH, N, d, block_size), exceeds
+ * BSA_TOPK_STATIC_SCRATCH_BYTES (that is BH * M * d > 262144) returns
+ * BSA_ERR_BUFFER_TOO_SMALL before any CUDA call, with nothing launched and
+ * the outputs untouched; use bsa_topk_pattern with a workspace instead.
+ * BSA_ERR_CUDA if the symbol lookup or a launch fails; BSA_ERR_UNSUPPORTED
+ * for a device ordinal of 64 or more.
+ *
+ * Nothing needs to start at zero: neither the scratch (each call writes every
+ * element it reads before reading it) nor row_ptr / col_idx.
+ * Calls that overlap in time on one device -- on different streams, or from
+ * host threads without an order between them -- share the one scratch array
+ * and race; order them (one stream, or events).
+ */
+#define BSA_TOPK_STATIC_SCRATCH_BYTES (4u * 1024u * 1024u)
+int bsa_topk_pattern_static(const void* Q, const void* K, int BH, int N, int d, int block_size,
+                            int top_k, int causal, int32_t* row_ptr, int32_t* col_idx,
+                            void* stream);
+
+/*
  * bsa_device_status -- read (and with clear != 0, reset) the status word of
  * the current device.  Synchronises the device.  Returns BSA_OK or
  * BSA_ERR_CUDA; *status receives an OR of BSA_STATUS_* bits accumulated by
