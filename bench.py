@@ -56,6 +56,7 @@ NCU_TRAFFIC = {
     "local_global_8k": (293797376 + 48656896, "cab8e846fd2d847e"),
     "bernoulli_4k": (201550592 + 51967488, "cab8e846fd2d847e"),
     "causal_loglinear_32k": (806639360 + 254766848, "cab8e846fd2d847e"),
+    "topk_4k": (25480704, "cab8e846fd2d847e"),
 }
 
 

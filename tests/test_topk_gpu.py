@@ -37,6 +37,10 @@ CASES = [
     (1, 2, 4096, 64, 32, 25, False),   # 20 % of 128 blocks
     (1, 1, 64, 64, 64, 0, False),      # M = 1
     (1, 1, 512, 64, 32, 100, True),    # top_k beyond the row: every allowed block
+    # more heads and rows; M = 120 and 60 pad the sort to 128 and 64 entries
+    (1, 12, 3840, 64, 32, 10, True),
+    (2, 5, 2048, 64, 32, 7, False),
+    (1, 5, 3840, 128, 64, 3, True),
 ]
 
 
