@@ -9,6 +9,9 @@ CUDA extension fails loudly when it is missing instead of falling back here.
   "Block Sparse Attention with Log-Linear Complexity", section 3.3: a softmax
   restricted to the connected key blocks, then the weighted sum of V).
 * ``patterns.py`` -- the block patterns enumerated from the pages' rules.
+* ``topk.py`` -- content-based top-k block selection.
+* ``decode.py`` -- one decode step: a new token per (b, h) against the
+  cached tokens of its block row.
 
 Every function here is pinned by the ``-m "not gpu"`` tests against brute
 force, closed forms, library routines and a hand-enumerated block list; see

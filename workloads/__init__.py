@@ -168,3 +168,77 @@ def make_qkv_shape(B: int, H: int, N: int, d: int, seed: int, key_scale_max: flo
                  key_scale_max=key_scale_max)
     return make_qkv(w)
 
+
+
+# ---------------------------------------------------------------- decode
+# One decode step per (b, h): a new query token at position seq_len[b] - 1
+# attends to the cached tokens of the blocks its block row lists (the KV
+# cache in the (B, H, L, D) layout of "Block Sparse Attention with Log-Linear
+# Complexity", section 5.1).  The cache holds L tokens of room; seq_len draws
+# a ragged batch of filled lengths.
+
+@dataclasses.dataclass(frozen=True)
+class DecodeWorkload:
+    name: str
+    B: int
+    H: int
+    L: int                  # cache capacity in tokens
+    d: int
+    block_size: int
+    pattern: PatternDesc    # over M = L // block_size block rows
+    seed: int
+    min_len: int            # seq_len[b] drawn uniformly from [min_len, L]
+    append: bool = True     # the step writes the new token's k and v into the cache
+
+    @property
+    def M(self) -> int:
+        return self.L // self.block_size
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / math.sqrt(self.d)
+
+
+DECODE_WORKLOADS = {
+    # 8 sequences of 16K-32K tokens, 32 heads, d=128, block 128: the causal
+    # log-linear pattern of causal_loglinear_32k (strides k=0..7, anchors
+    # {0,128,255}) read by one new token per (b, h)
+    "decode_loglinear_32k": DecodeWorkload(
+        "decode_loglinear_32k", 8, 32, 32768, 128, 128, _loglinear(256, 32, 7, causal=True),
+        seed=9, min_len=16384),
+    # a small one for parity: 4 sequences of 1..4096 tokens, block 32, d=64
+    "decode_loglinear_4k": DecodeWorkload(
+        "decode_loglinear_4k", 4, 16, 4096, 64, 32, _loglinear(128, 16, 6, causal=True),
+        seed=10, min_len=1),
+}
+
+
+def make_decode_inputs(w: DecodeWorkload, device="cpu", seed: Optional[int] = None):
+    """Seeded decode inputs on `device` (a torch generator of that device).
+
+    Draw order: seq_len [B] int32 uniform in [min_len, L]; q, k_new, v_new
+    [B, H, d]; then the K cache and the V cache [B, H, L, d], one batch entry
+    at a time; all fp32 randn cast to bf16.  Cache rows at and beyond
+    seq_len[b] - 1 hold random values too (stale entries of a reused cache).
+    Returns (q, k_new, v_new, k_cache, v_cache, seq_len).
+    """
+    import torch
+
+    g = torch.Generator(device=device)
+    g.manual_seed(w.seed if seed is None else seed)
+    lens = torch.randint(w.min_len, w.L + 1, (w.B,), generator=g, device=device,
+                         dtype=torch.int64).to(torch.int32)
+
+    def bf16(shape):
+        return torch.randn(shape, generator=g, device=device, dtype=torch.float32).to(torch.bfloat16)
+
+    q = bf16((w.B, w.H, w.d))
+    k_new = bf16((w.B, w.H, w.d))
+    v_new = bf16((w.B, w.H, w.d))
+    caches = []
+    for _ in range(2):
+        c = torch.empty((w.B, w.H, w.L, w.d), dtype=torch.bfloat16, device=device)
+        for b in range(w.B):
+            c[b] = bf16((w.H, w.L, w.d))
+        caches.append(c)
+    return q, k_new, v_new, caches[0], caches[1], lens
