@@ -57,6 +57,8 @@ NCU_TRAFFIC = {
     "bernoulli_4k": (201550592 + 51967488, "cab8e846fd2d847e"),
     "causal_loglinear_32k": (806639360 + 254766848, "cab8e846fd2d847e"),
     "topk_4k": (25480704, "cab8e846fd2d847e"),
+    # the decode kernel, keyed by the hash of DECODE_SOURCES
+    "decode_loglinear_32k": (175425792 + 3372544, "7be0c4ee875188a6"),
 }
 
 
@@ -111,14 +113,15 @@ def compulsory_bytes(w) -> float:
     return 4.0 * w.B * w.H * w.N * w.d * 2 + 4.0 * w.B * w.H * w.N
 
 
-# The files the forward kernel is compiled from (bsa_forward.cu and what it includes).
+# The files each kernel is compiled from (its .cu and what it includes).
 FORWARD_SOURCES = ("bsa_common.cuh", "bsa_forward.cu", "bsa_fwd_rows.cuh", "sm100_ptx.cuh")
+DECODE_SOURCES = ("bsa_decode.cu", "sm100_ptx.cuh")
 
 
-def kernel_hash() -> str:
-    """sha256 prefix over the forward kernel's source files (sorted by name)."""
+def kernel_hash(sources=FORWARD_SOURCES) -> str:
+    """sha256 prefix over a kernel's source files (sorted by name)."""
     h = hashlib.sha256()
-    for name in sorted(FORWARD_SOURCES):
+    for name in sorted(sources):
         with open(os.path.join(KERNEL_DIR, name), "rb") as f:
             h.update(name.encode() + b"\0" + f.read())
     return h.hexdigest()[:16]
@@ -256,6 +259,234 @@ def run_reference(args, w, rank, world):
                    "block_size": w_in.block_size},
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
                          "sample": f"{rows_done} random query rows of {w.name} over {args.steps} steps"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ decode
+def decode_tokens(w, lens, rp, ci) -> np.ndarray:
+    """Cached tokens each (b, h) attends to in one decode step, [B, H]: the
+    blocks j <= i of CSR row i = (seq_len - 1) // block_size, counted once,
+    block i only up to the new token."""
+    bs, M = w.block_size, w.M
+    n = np.zeros((w.B, w.H), dtype=np.int64)
+    for b in range(w.B):
+        t = int(lens[b]) - 1
+        i = t // bs
+        for h in range(w.H):
+            cols = set(int(j) for j in ci[rp[h * M + i]:rp[h * M + i + 1]])
+            n[b, h] = sum(bs for j in cols if j < i) + (t - i * bs + 1 if i in cols else 0)
+    return n
+
+
+def decode_flops(w, tokens) -> float:
+    return 4.0 * w.d * float(tokens.sum())
+
+
+def decode_bytes(w, tokens) -> float:
+    """Algorithmic HBM bytes of one step: the attended K and V rows; q, k_new
+    and v_new read; the appended K and V rows written; O, LSE and seq_len."""
+    per_token = 2.0 * w.d * 2
+    vectors = w.B * w.H * w.d * 2.0 * (3 + (2 if w.append else 0) + 1)
+    return per_token * float(tokens.sum()) + vectors + 4.0 * w.B * w.H + 4.0 * w.B
+
+
+def cpu_decode_sample(w, q, kn, vn, K, V, lens, rp, ci, seconds: float, rng_seed: int = 0):
+    """Time the fp64 decode oracle on random (b, h) pairs (CPU tensors) until
+    `seconds` of work; returns (useful TFLOP/s, threads, pairs done, seconds)."""
+    from oracle import decode as odec
+
+    rng = np.random.default_rng(rng_seed)
+    tokens = decode_tokens(w, lens, rp, ci)
+    done, flops, elapsed, batch = 0, 0.0, 0.0, 4
+    while elapsed < seconds:
+        pairs = [(int(b), int(h)) for b, h in zip(rng.integers(0, w.B, batch),
+                                                  rng.integers(0, w.H, batch))]
+        t0 = time.perf_counter()
+        odec.decode(q, K, V, lens, rp, ci, w.block_size, w.scale,
+                    k_new=kn if w.append else None, v_new=vn if w.append else None, pairs=pairs)
+        elapsed += time.perf_counter() - t0
+        flops += sum(4.0 * w.d * tokens[b, h] for b, h in pairs)
+        done += batch
+        if elapsed < seconds / 8:
+            batch *= 2
+    import torch
+
+    return flops / elapsed / 1e12, torch.get_num_threads(), done, elapsed
+
+
+def run_decode(args, w, rank, world, local_rank):
+    import torch
+
+    import block_sparse_attention_38_b200 as bsa
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    bsa.library()
+    q, kn, vn, K, V, lens = workloads.make_decode_inputs(w, device=dev, seed=replica_seed(w, rank))
+    rp_np, ci_np = bsa.build_pattern_from(w.pattern)
+    rp = torch.from_numpy(rp_np).to(dev)
+    ci = torch.from_numpy(ci_np).to(dev)
+    lens_np = lens.cpu().numpy()
+    tokens = decode_tokens(w, lens_np, rp_np, ci_np)
+    flops, nbytes = decode_flops(w, tokens), decode_bytes(w, tokens)
+    O = torch.empty((w.B, w.H, w.d), dtype=torch.bfloat16, device=dev)
+    L = torch.empty((w.B, w.H), dtype=torch.float32, device=dev)
+    flush = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    kw = dict(k_new=kn, v_new=vn) if w.append else {}
+
+    def step():
+        bsa.decode(q, K, V, lens, rp, ci, w.block_size, w.scale, out=O, lse=L, **kw)
+
+    for _ in range(args.warmup):
+        flush.fill_(1)
+        step()
+    torch.cuda.synchronize()
+    bsa.decode_status(clear=True)
+    visible = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+    ids = [x.strip() for x in visible.split(",") if x.strip()]
+    clocks = ClockSampler(ids[local_rank] if local_rank < len(ids) else str(local_rank))
+    if rank == 0:
+        clocks.start()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush.fill_(i & 0xFF)
+        starts[i].record(stream)
+        step()
+        ends[i].record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clock_info = clocks.stop() if rank == 0 else None
+    per_step = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    total_ms = float(sum(per_step))
+    status = bsa.decode_status(clear=True)
+    if status:
+        raise RuntimeError(f"decode kernel reported device status {status:#x}")
+
+    # End to end through the public API: the KV cache is device state; each
+    # step brings the new token's q, k, v and the lengths from pinned host
+    # memory, runs the step and returns O and LSE to pinned host memory.
+    qp, knp, vnp = (t.cpu().pin_memory() for t in (q, kn, vn))
+    lp = lens.cpu().pin_memory()
+    Oh = torch.empty(O.shape, dtype=O.dtype).pin_memory()
+    Lh = torch.empty(L.shape, dtype=L.dtype).pin_memory()
+    qd, knd, vnd, ld = (torch.empty_like(t) for t in (q, kn, vn, lens))
+    ins = [(qd, qp), (ld, lp)] + ([(knd, knp), (vnd, vnp)] if w.append else [])
+    h2d = sum(src.numel() * src.element_size() for _, src in ins)
+    d2h = Oh.numel() * Oh.element_size() + Lh.numel() * Lh.element_size()
+    ekw = dict(k_new=knd, v_new=vnd) if w.append else {}
+
+    def e2e_step():
+        for dst, src in ins:
+            dst.copy_(src, non_blocking=True)
+        bsa.decode(qd, K, V, ld, rp, ci, w.block_size, w.scale, out=O, lse=L, **ekw)
+        Oh.copy_(O, non_blocking=True)
+        Lh.copy_(L, non_blocking=True)
+
+    for _ in range(max(1, args.warmup)):
+        e2e_step()
+    torch.cuda.synchronize()
+    e_steps = max(3, min(args.steps, 50))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / e_steps
+    if bsa.decode_status(clear=True):
+        raise RuntimeError("decode kernel reported a device status in the end-to-end leg")
+    if not torch.equal(Oh, O.cpu()):
+        raise RuntimeError("end-to-end result differs from the device result")
+
+    total_ms, e2e_ms = max_over_ranks([total_ms, e2e_ms], world, device=dev)
+    if rank != 0:
+        return
+    ms = total_ms / args.steps
+    peaks, peak_src = load_peaks()
+    peak_tc = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    peak_hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    t_tc = flops / (peak_tc * 1e12)
+    t_hbm = nbytes / (peak_hbm * 1e9)
+    roof = {"bound": "hbm", "achieved": nbytes / (ms * 1e-3) / 1e9, "peak": peak_hbm,
+            "unit": "GB/s"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    tr = NCU_TRAFFIC.get(w.name)
+    roof["traffic"] = tr[0] if tr and tr[1] == kernel_hash(DECODE_SOURCES) else None
+    roof["peak_source"] = f"{peak_src} (MEASURED_PEAKS.json burst)" if peak_src == "measured" else "fallback"
+    roof["roofline_frac_max_of_tc_hbm"] = max(t_tc, t_hbm) / (ms * 1e-3)
+    roof["kernel"] = "bsa::decode::decode_kernel"
+    roof["kernel_ms"] = ms
+    roof["algorithmic_bytes"] = nbytes
+
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        Kc, Vc = K.cpu(), V.cpu()
+        tf, threads, npairs, el = cpu_decode_sample(w, q.cpu(), kn.cpu(), vn.cpu(), Kc, Vc,
+                                                    lens_np, rp_np, ci_np, args.cpu_seconds)
+        cpu = {"value": tf, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+               "sample": f"{npairs} random (b, h) decode queries of {w.name} ({el:.1f} s, fp64)"}
+    line = {
+        "metric": METRIC, "value": whole_job_tflops(flops, world, ms), "unit": "TFLOP/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "L": w.L, "d": w.d,
+                   "block_size": w.block_size, "tokens_attended": int(tokens.sum()),
+                   "append": bool(w.append),
+                   "l2": "flushed before every timed step (512 MB write)",
+                   "parallelism": f"replicas x{world}"},
+        "roofline": roof,
+        "cpu_baseline": cpu,
+        "e2e": {"value": whole_job_tflops(flops, world, e2e_ms), "unit": "TFLOP/s",
+                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+                "ms_per_step": e2e_ms},
+        "gpu_launches": args.steps,
+        "clocks": clock_info,
+        "min_ms": min(per_step), "median_ms": statistics.median(per_step),
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_reference_decode(args, w, rank, world):
+    """fp64 CPU decode oracle on the host cores, each step a bounded sample of (b, h)."""
+    if rank != 0:
+        return
+    from oracle import patterns
+
+    q, kn, vn, K, V, lens = workloads.make_decode_inputs(w, device="cpu")
+    rp, ci = patterns.csr(w.pattern)
+    lens_np = lens.numpy()
+    for i in range(args.warmup):
+        cpu_decode_sample(w, q, kn, vn, K, V, lens_np, rp, ci, 0.2, rng_seed=1000 + i)
+    vals, times, done, threads = [], [], 0, 0
+    for i in range(args.steps):
+        tf, threads, n, el = cpu_decode_sample(w, q, kn, vn, K, V, lens_np, rp, ci, 2.0, rng_seed=i)
+        vals.append(tf)
+        times.append(el)
+        done += n
+    value = statistics.median(vals)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * statistics.mean(times), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "L": w.L, "d": w.d,
+                   "block_size": w.block_size},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                         "sample": f"{done} random (b, h) decode queries of {w.name} over {args.steps} steps"},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -486,19 +717,22 @@ def main():
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=list(workloads.WORKLOADS))
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD,
+                    choices=list(workloads.WORKLOADS) + list(workloads.DECODE_WORKLOADS))
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
-    w = workloads.WORKLOADS[args.workload]
+    decode = args.workload in workloads.DECODE_WORKLOADS
+    w = (workloads.DECODE_WORKLOADS if decode else workloads.WORKLOADS)[args.workload]
+    run = run_decode if decode else run_ours
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
-        run_reference(args, w, rank, world)
+        (run_reference_decode if decode else run_reference)(args, w, rank, world)
         return
     if world > 1:
         import datetime
@@ -509,11 +743,11 @@ def main():
         torch.cuda.set_device(local_rank)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
         try:
-            run_ours(args, w, rank, world, local_rank)
+            run(args, w, rank, world, local_rank)
         finally:
             dist.destroy_process_group()
     else:
-        run_ours(args, w, 0, 1, 0)
+        run(args, w, 0, 1, 0)
 
 
 if __name__ == "__main__":

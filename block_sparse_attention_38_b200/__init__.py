@@ -47,6 +47,7 @@ BIGBIRD = 4
 STATUS_TIMEOUT = 0x1
 STATUS_BAD_COLUMN = 0x2
 STATUS_BAD_ROW_PTR = 0x4
+STATUS_BAD_SEQ_LEN = 0x8
 
 
 class BsaError(RuntimeError):
@@ -95,6 +96,10 @@ def library() -> ctypes.CDLL:
         lib.bsa_topk_pattern.restype = ctypes.c_int
         lib.bsa_topk_pattern.argtypes = [vp, vp] + [ctypes.c_int] * 6 + [vp, vp, vp,
                                                                           ctypes.c_size_t, vp]
+        lib.bsa_decode.restype = ctypes.c_int
+        lib.bsa_decode.argtypes = [vp] * 8 + [ctypes.c_int] * 5 + [ctypes.c_float, vp, vp, vp]
+        lib.bsa_decode_status.restype = ctypes.c_int
+        lib.bsa_decode_status.argtypes = [ctypes.POINTER(ctypes.c_uint32), ctypes.c_int]
         lib.bsa_topk_pattern_static.restype = ctypes.c_int
         lib.bsa_topk_pattern_static.argtypes = [vp, vp] + [ctypes.c_int] * 6 + [vp, vp, vp]
         _lib = lib
@@ -265,6 +270,63 @@ def topk_pattern_static(q, k, block_size: int, top_k: int, causal: bool, row_ptr
                            f"static scratch holds {TOPK_STATIC_SCRATCH_BYTES})")
     _check(rc, "bsa_topk_pattern_static")
     return row_ptr, col_idx[:nnz]
+
+
+def decode(q, k_cache, v_cache, seq_len, row_ptr, col_idx, block_size: int, scale: float,
+           k_new=None, v_new=None, out=None, lse=None):
+    """One decode step (bsa_decode) on q's device and current stream.
+
+    q: CUDA bf16 [B, H, d]; k_cache, v_cache: CUDA bf16 [B, H, L, d] (with
+    k_new / v_new [B, H, d] given, row seq_len[b] - 1 of each cache is
+    overwritten with them first); seq_len: CUDA int32 [B]; row_ptr, col_idx:
+    CUDA int32 block-CSR over L // block_size block rows per head.  Returns
+    (O bf16 [B, H, d], LSE fp32 [B, H]).
+    """
+    import torch
+
+    lib = library()
+    if q.dim() != 3 or k_cache.dim() != 4 or v_cache.shape != k_cache.shape:
+        raise ValueError("q must be [B, H, d] and the caches [B, H, L, d]")
+    B, H, L, d = (int(x) for x in k_cache.shape)
+    if tuple(q.shape) != (B, H, d):
+        raise ValueError("q must be [B, H, d] with the caches' B, H, d")
+    named = [("q", q), ("k_cache", k_cache), ("v_cache", v_cache)]
+    if (k_new is None) != (v_new is None):
+        raise ValueError("give both k_new and v_new, or neither")
+    if k_new is not None:
+        named += [("k_new", k_new), ("v_new", v_new)]
+        if tuple(k_new.shape) != (B, H, d) or tuple(v_new.shape) != (B, H, d):
+            raise ValueError("k_new, v_new must be [B, H, d]")
+    for name, t in named:
+        if not t.is_cuda or t.dtype != torch.bfloat16 or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous CUDA bf16 tensor")
+        if t.device != q.device:
+            raise ValueError(f"{name} must be on q's device")
+    for name, t in (("seq_len", seq_len), ("row_ptr", row_ptr), ("col_idx", col_idx)):
+        if not t.is_cuda or t.dtype != torch.int32 or not t.is_contiguous() or t.device != q.device:
+            raise ValueError(f"{name} must be a contiguous int32 tensor on q's device")
+    if seq_len.numel() != B:
+        raise ValueError("seq_len must hold B entries")
+    if row_ptr.numel() != H * (L // int(block_size)) + 1:
+        raise ValueError("row_ptr must have H*M+1 entries")
+    O = torch.empty((B, H, d), dtype=torch.bfloat16, device=q.device) if out is None else out
+    LSE = torch.empty((B, H), dtype=torch.float32, device=q.device) if lse is None else lse
+    with torch.cuda.device(q.device):
+        stream = torch.cuda.current_stream(q.device).cuda_stream
+        rc = lib.bsa_decode(q.data_ptr(), None if k_new is None else k_new.data_ptr(),
+                            None if v_new is None else v_new.data_ptr(), k_cache.data_ptr(),
+                            v_cache.data_ptr(), row_ptr.data_ptr(), col_idx.data_ptr(),
+                            seq_len.data_ptr(), B, H, L, d, int(block_size), float(scale),
+                            O.data_ptr(), LSE.data_ptr(), stream)
+    _check(rc, "bsa_decode")
+    return O, LSE
+
+
+def decode_status(clear: bool = True) -> int:
+    """OR of STATUS_* bits raised by the decode kernel on the current device (synchronises it)."""
+    v = ctypes.c_uint32(0)
+    _check(library().bsa_decode_status(ctypes.byref(v), int(bool(clear))), "bsa_decode_status")
+    return int(v.value)
 
 
 def device_status(clear: bool = True) -> int:

@@ -156,6 +156,7 @@ int bsa_forward(const void* Q, const void* K, const void* V,
 #define BSA_STATUS_TIMEOUT     0x1u  /* a bounded wait inside the kernel gave up */
 #define BSA_STATUS_BAD_COLUMN  0x2u  /* a column index outside [0, M) was skipped */
 #define BSA_STATUS_BAD_ROW_PTR 0x4u  /* row_ptr[i+1] < row_ptr[i] was seen; the row was treated as empty */
+#define BSA_STATUS_BAD_SEQ_LEN 0x8u  /* bsa_decode: a seq_len outside [1, L]; that entry was treated as empty */
 
 /*
  * Content-based top-k block selection (a pattern computed from Q and K on the
@@ -232,6 +233,45 @@ int bsa_topk_pattern(const void* Q, const void* K, int BH, int N, int d, int blo
 int bsa_topk_pattern_static(const void* Q, const void* K, int BH, int N, int d, int block_size,
                             int top_k, int causal, int32_t* row_ptr, int32_t* col_idx,
                             void* stream);
+
+/*
+ * bsa_decode -- one decode step of block-sparse attention over a KV cache.
+ *
+ * "Block Sparse Attention with Log-Linear Complexity" keeps the KV cache in
+ * the (B, H, N, D) layout of past_key_values (section 5.1) and claims the
+ * pattern cuts cache traffic at inference (section 1).  For each (b, h), the
+ * new token sits at position t = seq_len[b] - 1, in block row i = t /
+ * block_size.  It attends to the cached tokens of the blocks j <= i listed
+ * in CSR row i of head h: all block_size tokens of a block j < i, the tokens
+ * i*block_size .. t of block i (blocks j > i hold no cached tokens yet and are
+ * skipped).  O = sum softmax(scale * q.k) v; LSE = the natural log-sum-exp of
+ * the scaled scores; no tokens gives O = 0 and LSE = -inf.  A row is a set
+ * (repeated columns count once).
+ *
+ * q: bf16 [B, H, d]; k_new, v_new: bf16 [B, H, d], or both NULL; k_cache,
+ * v_cache: bf16 [B, H, L, d] contiguous.  With k_new/v_new given the step
+ * first writes them into cache row t of each (b, h) -- the append of the new
+ * token -- and attends to them there; otherwise row t must already hold the
+ * new token.  Rows after t are never read.  row_ptr int32 [H*M+1] and
+ * col_idx int32: the forward's block-CSR over M = L / block_size block rows.
+ * seq_len: device int32 [B], cached tokens including the new one, 1..L.
+ * O: bf16 [B, H, d]; LSE: fp32 [B, H].  All pointers are caller-owned
+ * device memory, 16-byte aligned (LSE 4-byte); the call is enqueued on
+ * `stream` and allocates nothing.
+ * Supported: d in {64, 128}; block_size in {32, 64, 128}; L % block_size ==
+ * 0; M <= 4096.  Else BSA_ERR_INVALID_ARG / BSA_ERR_UNSUPPORTED with nothing
+ * launched; BSA_ERR_CUDA if the launch fails.  Device-side checks (a
+ * seq_len outside [1, L], a column outside [0, M), a decreasing row_ptr, a
+ * timed-out wait) set BSA_STATUS_* bits read by bsa_decode_status.
+ */
+int bsa_decode(const void* q, const void* k_new, const void* v_new, void* k_cache,
+               void* v_cache, const int32_t* row_ptr, const int32_t* col_idx,
+               const int32_t* seq_len, int B, int H, int L, int d, int block_size,
+               float scale, void* O, float* LSE, void* stream);
+
+/* bsa_decode_status -- as bsa_device_status, for the status word the decode
+ * kernel sets (BSA_STATUS_TIMEOUT, _BAD_COLUMN, _BAD_ROW_PTR, _BAD_SEQ_LEN). */
+int bsa_decode_status(uint32_t* status, int clear);
 
 /*
  * bsa_device_status -- read (and with clear != 0, reset) the status word of
