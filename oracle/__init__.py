@@ -12,6 +12,8 @@ CUDA extension fails loudly when it is missing instead of falling back here.
 * ``topk.py`` -- content-based top-k block selection.
 * ``decode.py`` -- one decode step: a new token per (b, h) against the
   cached tokens of its block row.
+* ``backward.py`` -- the gradients dQ, dK, dV of the forward, and the
+  column-major copy of a block-CSR.
 
 Every function here is pinned by the ``-m "not gpu"`` tests against brute
 force, closed forms, library routines and a hand-enumerated block list; see
