@@ -96,6 +96,17 @@ def library() -> ctypes.CDLL:
         lib.bsa_topk_pattern.restype = ctypes.c_int
         lib.bsa_topk_pattern.argtypes = [vp, vp] + [ctypes.c_int] * 6 + [vp, vp, vp,
                                                                           ctypes.c_size_t, vp]
+        lib.bsa_transpose_pattern.restype = ctypes.c_int
+        lib.bsa_transpose_pattern.argtypes = [vp, vp, i32, i32, vp, vp, i64,
+                                              ctypes.POINTER(ctypes.c_int64)]
+        lib.bsa_backward_workspace_bytes.restype = ctypes.c_size_t
+        lib.bsa_backward_workspace_bytes.argtypes = [ctypes.c_int] * 3
+        lib.bsa_backward.restype = ctypes.c_int
+        lib.bsa_backward.argtypes = [vp] * 10 + [ctypes.c_int] * 5 + [ctypes.c_float, ctypes.c_int,
+                                                                    vp, vp, vp, vp,
+                                                                    ctypes.c_size_t, vp]
+        lib.bsa_backward_status.restype = ctypes.c_int
+        lib.bsa_backward_status.argtypes = [ctypes.POINTER(ctypes.c_uint32), ctypes.c_int]
         lib.bsa_decode.restype = ctypes.c_int
         lib.bsa_decode.argtypes = [vp] * 8 + [ctypes.c_int] * 5 + [ctypes.c_float, vp, vp, vp]
         lib.bsa_decode_status.restype = ctypes.c_int
@@ -270,6 +281,72 @@ def topk_pattern_static(q, k, block_size: int, top_k: int, causal: bool, row_ptr
                            f"static scratch holds {TOPK_STATIC_SCRATCH_BYTES})")
     _check(rc, "bsa_topk_pattern_static")
     return row_ptr, col_idx[:nnz]
+
+
+def transpose_pattern(row_ptr, col_idx, H: int, M: int) -> Tuple[np.ndarray, np.ndarray]:
+    """Column-major copy of a host block-CSR (bsa_transpose_pattern): (col_ptr, row_idx)."""
+    lib = library()
+    rp = np.ascontiguousarray(row_ptr, dtype=np.int32)
+    ci = np.ascontiguousarray(col_idx, dtype=np.int32)
+    if rp.size != int(H) * int(M) + 1:
+        raise ValueError("row_ptr must have H*M+1 entries")
+    cp = np.empty(rp.size, dtype=np.int32)
+    ri = np.empty(max(int(rp[-1]), 1), dtype=np.int32)
+    nnz = ctypes.c_int64(0)
+    _check(lib.bsa_transpose_pattern(rp.ctypes.data, ci.ctypes.data if ci.size else None, int(H),
+                                     int(M), cp.ctypes.data, ri.ctypes.data, ri.size,
+                                     ctypes.byref(nnz)), "bsa_transpose_pattern")
+    return cp, ri[:nnz.value].copy()
+
+
+def backward(q, k, v, o, do, lse, row_ptr, col_idx, col_ptr, row_idx, block_size: int,
+             scale: float, causal: bool = False, workspace=None):
+    """Gradients of `forward` (bsa_backward) on q's device and current stream.
+
+    q, k, v, o, do: CUDA bf16 [B, H, N, d] contiguous (o, lse from `forward`);
+    lse: CUDA fp32 [B, H, N]; row_ptr / col_idx: the forward's CSR and
+    col_ptr / row_idx its `transpose_pattern`, all CUDA int32.  Returns
+    (dQ, dK, dV) as CUDA bf16 [B, H, N, d].
+    """
+    import torch
+
+    lib = library()
+    if q.dim() != 4:
+        raise ValueError("q must be [B, H, N, d]")
+    B, H, N, d = (int(x) for x in q.shape)
+    for name, t in (("q", q), ("k", k), ("v", v), ("o", o), ("do", do)):
+        if tuple(t.shape) != (B, H, N, d):
+            raise ValueError(f"{name} must have q's shape")
+        if not t.is_cuda or t.dtype != torch.bfloat16 or not t.is_contiguous() or t.device != q.device:
+            raise ValueError(f"{name} must be a contiguous CUDA bf16 tensor on q's device")
+    if (tuple(lse.shape) != (B, H, N) or lse.dtype != torch.float32 or not lse.is_contiguous()
+            or lse.device != q.device):
+        raise ValueError("lse must be a contiguous fp32 [B, H, N] tensor on q's device")
+    for name, t in (("row_ptr", row_ptr), ("col_idx", col_idx), ("col_ptr", col_ptr),
+                    ("row_idx", row_idx)):
+        if not t.is_cuda or t.dtype != torch.int32 or not t.is_contiguous() or t.device != q.device:
+            raise ValueError(f"{name} must be a contiguous int32 tensor on q's device")
+    nbytes = int(lib.bsa_backward_workspace_bytes(B, H, N))
+    if workspace is None:
+        workspace = torch.empty(max(nbytes // 4, 1), dtype=torch.float32, device=q.device)
+    dq, dk, dv = (torch.empty_like(q) for _ in range(3))
+    with torch.cuda.device(q.device):
+        stream = torch.cuda.current_stream(q.device).cuda_stream
+        rc = lib.bsa_backward(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(),
+                              lse.data_ptr(), row_ptr.data_ptr(), col_idx.data_ptr(),
+                              col_ptr.data_ptr(), row_idx.data_ptr(), B, H, N, d, int(block_size),
+                              float(scale), int(bool(causal)), dq.data_ptr(), dk.data_ptr(),
+                              dv.data_ptr(), workspace.data_ptr(),
+                              workspace.numel() * workspace.element_size(), stream)
+    _check(rc, "bsa_backward")
+    return dq, dk, dv
+
+
+def backward_status(clear: bool = True) -> int:
+    """OR of STATUS_* bits raised by the backward kernels on the current device (synchronises it)."""
+    v = ctypes.c_uint32(0)
+    _check(library().bsa_backward_status(ctypes.byref(v), int(bool(clear))), "bsa_backward_status")
+    return int(v.value)
 
 
 def decode(q, k_cache, v_cache, seq_len, row_ptr, col_idx, block_size: int, scale: float,

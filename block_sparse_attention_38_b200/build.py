@@ -18,7 +18,8 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 SOURCES = [os.path.join(CSRC, "bsa_pattern.cpp"), os.path.join(CSRC, "bsa_forward.cu"),
-           os.path.join(CSRC, "bsa_topk.cu"), os.path.join(CSRC, "bsa_decode.cu")]
+           os.path.join(CSRC, "bsa_topk.cu"), os.path.join(CSRC, "bsa_decode.cu"),
+           os.path.join(CSRC, "bsa_backward.cu")]
 DEPS = SOURCES + [os.path.join(CSRC, f) for f in sorted(os.listdir(CSRC)) if f.endswith(".cuh")] + [
     os.path.join(ROOT, "include", "bsa.h")]
 LIB = os.path.join(HERE, "libbsa.so")

@@ -192,4 +192,52 @@ extern "C" int bsa_validate_pattern(const int32_t* row_ptr, const int32_t* col_i
   return BSA_OK;
 }
 
+// Column-major copy of a block-CSR (the backward's dK/dV walk): for each
+// (h, column j), the block rows i listing j, ascending; a column repeated
+// within a row counts once.  Two passes: count, then fill.
+extern "C" int bsa_transpose_pattern(const int32_t* row_ptr, const int32_t* col_idx, int32_t H,
+                                     int32_t M, int32_t* col_ptr, int32_t* row_idx,
+                                     int64_t cap, int64_t* nnz_out) {
+  if (row_ptr == nullptr || col_ptr == nullptr || nnz_out == nullptr || H < 1 || M < 1 ||
+      cap < 0)
+    return BSA_ERR_INVALID_ARG;
+  const int64_t rows = int64_t(H) * M;
+  if (row_ptr[0] != 0) return BSA_ERR_BAD_PATTERN;
+  for (int64_t r = 0; r < rows; ++r)
+    if (row_ptr[r + 1] < row_ptr[r]) return BSA_ERR_BAD_PATTERN;
+  if (row_ptr[rows] > 0 && col_idx == nullptr) return BSA_ERR_INVALID_ARG;
+  std::vector<int64_t> count(static_cast<size_t>(rows) + 1, 0);
+  for (int64_t e = 0; e < row_ptr[rows]; ++e)
+    if (col_idx[e] < 0 || col_idx[e] >= M) return BSA_ERR_BAD_PATTERN;
+  // count, with a per-row stamp so that repeats within a row count once
+  std::vector<int32_t> stamp(static_cast<size_t>(M), -1);  // last row that listed column j
+  for (int64_t r = 0; r < rows; ++r) {
+    const int64_t h = r / M;
+    for (int32_t p = row_ptr[r]; p < row_ptr[r + 1]; ++p) {
+      const int32_t j = col_idx[p];
+      if (stamp[j] == static_cast<int32_t>(r)) continue;
+      stamp[j] = static_cast<int32_t>(r);
+      ++count[static_cast<size_t>(h * M + j) + 1];
+    }
+  }
+  for (int64_t c = 0; c < rows; ++c) count[c + 1] += count[c];
+  *nnz_out = count[static_cast<size_t>(rows)];
+  if (count[static_cast<size_t>(rows)] > cap) return BSA_ERR_BUFFER_TOO_SMALL;
+  if (count[static_cast<size_t>(rows)] > INT32_MAX) return BSA_ERR_UNSUPPORTED;
+  if (count[static_cast<size_t>(rows)] > 0 && row_idx == nullptr) return BSA_ERR_INVALID_ARG;
+  std::vector<int64_t> fill(count.begin(), count.end() - 1);
+  std::fill(stamp.begin(), stamp.end(), -1);
+  for (int64_t r = 0; r < rows; ++r) {  // rows in ascending order: each column list ascends
+    const int64_t h = r / M;
+    for (int32_t p = row_ptr[r]; p < row_ptr[r + 1]; ++p) {
+      const int32_t j = col_idx[p];
+      if (stamp[j] == static_cast<int32_t>(r)) continue;
+      stamp[j] = static_cast<int32_t>(r);
+      row_idx[fill[static_cast<size_t>(h * M + j)]++] = static_cast<int32_t>(r - h * M);
+    }
+  }
+  for (int64_t c = 0; c <= rows; ++c) col_ptr[c] = static_cast<int32_t>(count[static_cast<size_t>(c)]);
+  return BSA_OK;
+}
+
 extern "C" int bsa_version(void) { return 101; }

@@ -235,6 +235,57 @@ int bsa_topk_pattern_static(const void* Q, const void* K, int BH, int N, int d, 
                             void* stream);
 
 /*
+ * bsa_transpose_pattern -- column-major copy of a block-CSR, for the
+ * backward's dK/dV walk (host only, integer work).  For every (h, column j)
+ * col_ptr[h*M + j] .. col_ptr[h*M + j + 1] indexes row_idx, the block rows
+ * i that list j, ascending; a column repeated within a row counts once.
+ * row_ptr [H*M+1], col_idx: host arrays of a CSR; col_ptr: host int32
+ * [H*M+1]; row_idx: host int32 of capacity `cap` (at most row_ptr[H*M]
+ * entries are written).  *nnz_out receives the entry count, also when it
+ * exceeds cap (then BSA_ERR_BUFFER_TOO_SMALL, nothing written).
+ * BSA_ERR_BAD_PATTERN for a decreasing row_ptr, row_ptr[0] != 0 or a column
+ * outside [0, M); BSA_ERR_INVALID_ARG for null pointers or H, M < 1.
+ */
+int bsa_transpose_pattern(const int32_t* row_ptr, const int32_t* col_idx, int32_t H, int32_t M,
+                          int32_t* col_ptr, int32_t* row_idx, int64_t cap, int64_t* nnz_out);
+
+/* Device workspace bytes bsa_backward needs (D = dO . O per query row, fp32):
+ * 4 * B * H * N; 0 for invalid sizes. */
+size_t bsa_backward_workspace_bytes(int B, int H, int N);
+
+/*
+ * bsa_backward -- gradients of bsa_forward: dQ, dK, dV.
+ *
+ * "Block Sparse Attention with Log-Linear Complexity" notes that the sparse
+ * product falls back to dense work in the backward pass (section 4.2) and
+ * trains with the pattern (section 5.3).  With P_qk = exp(scale q.k - LSE_q)
+ * over the keys the forward allowed and D_q = dO_q . O_q:
+ * dV_k = sum_q P dO_q; dS = P (dO_q . v_k - D_q); dQ_q = scale sum_k dS k_k;
+ * dK_k = scale sum_q dS q_q.
+ *
+ * Q, K, V, O, dO: device bf16 [B, H, N, d] contiguous (O and LSE from
+ * bsa_forward on the same inputs and pattern); LSE: device fp32 [B, H, N].
+ * row_ptr / col_idx: the forward's block-CSR (device); col_ptr / row_idx: its
+ * column-major copy from bsa_transpose_pattern (device).  dQ, dK, dV: device
+ * bf16 [B, H, N, d], fully written.  workspace: device memory of at least
+ * bsa_backward_workspace_bytes(B, H, N) bytes, 16-byte aligned (overwritten).
+ * Enqueued on `stream` (three kernels); nothing allocated or synchronised.
+ * Supported: d in {64, 128}; block_size in {32, 64, 128}; N % 128 == 0;
+ * M <= 4096; 16-byte aligned tensors.  Else BSA_ERR_INVALID_ARG /
+ * BSA_ERR_UNSUPPORTED with nothing launched; BSA_ERR_BUFFER_TOO_SMALL for a
+ * short workspace; BSA_ERR_CUDA if a launch fails.  Device-side checks set
+ * BSA_STATUS_* bits read by bsa_backward_status.
+ */
+int bsa_backward(const void* Q, const void* K, const void* V, const void* O, const void* dO,
+                 const float* LSE, const int32_t* row_ptr, const int32_t* col_idx,
+                 const int32_t* col_ptr, const int32_t* row_idx, int B, int H, int N, int d,
+                 int block_size, float scale, int causal, void* dQ, void* dK, void* dV,
+                 void* workspace, size_t workspace_bytes, void* stream);
+
+/* bsa_backward_status -- as bsa_device_status, for the backward kernels' word. */
+int bsa_backward_status(uint32_t* status, int clear);
+
+/*
  * bsa_decode -- one decode step of block-sparse attention over a KV cache.
  *
  * "Block Sparse Attention with Log-Linear Complexity" keeps the KV cache in
