@@ -59,6 +59,9 @@ NCU_TRAFFIC = {
     "topk_4k": (25480704, "cab8e846fd2d847e"),
     # the decode kernel, keyed by the hash of DECODE_SOURCES
     "decode_loglinear_32k": (175425792 + 3372544, "7be0c4ee875188a6"),
+    # the backward's three kernels together (dot + dK/dV + dQ), one backward
+    "local_global_8k:backward": (134230272 + 3581696 + 340731392 + 115491072 + 333471744
+                                 + 55681792, "b99ddf4496188bae"),
 }
 
 
@@ -116,6 +119,7 @@ def compulsory_bytes(w) -> float:
 # The files each kernel is compiled from (its .cu and what it includes).
 FORWARD_SOURCES = ("bsa_common.cuh", "bsa_forward.cu", "bsa_fwd_rows.cuh", "sm100_ptx.cuh")
 DECODE_SOURCES = ("bsa_decode.cu", "sm100_ptx.cuh")
+BACKWARD_SOURCES = ("bsa_backward.cu", "sm100_ptx.cuh")
 
 
 def kernel_hash(sources=FORWARD_SOURCES) -> str:
@@ -260,6 +264,184 @@ def run_reference(args, w, rank, world):
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
                          "sample": f"{rows_done} random query rows of {w.name} over {args.steps} steps"},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------- backward
+ORACLE_BACKWARD_MAX_N = 8192  # the dense oracle's N x N fp64 arrays stay within a few GB
+
+
+def backward_flops(w, nnz_all_heads: int) -> float:
+    """Useful flops of one backward: per stored block the five products
+    S = QK^T, dP = dO V^T, dV = P^T dO, dQ = dS K, dK = dS^T Q (2 bs^2 d each)."""
+    return 10.0 * w.block_size * w.block_size * w.d * nnz_all_heads * w.B
+
+
+def backward_bytes(w) -> float:
+    """Compulsory bytes: Q, K, V, O, dO read, dQ, dK, dV written (bf16), LSE
+    read and D written and read (fp32)."""
+    return 8.0 * w.B * w.H * w.N * w.d * 2 + 3 * 4.0 * w.B * w.H * w.N
+
+
+def cpu_backward_sample(w, q, k, v, do, rp, ci, seconds: float, rng_seed: int = 0):
+    """Time the fp64 backward oracle on random (b, h) pairs until `seconds` of
+    work; returns (useful TFLOP/s, threads, pairs done, seconds)."""
+    import torch
+
+    from oracle import backward as obw
+
+    rng = np.random.default_rng(rng_seed)
+    M = w.M
+    done, flops, elapsed = 0, 0.0, 0.0
+    while elapsed < seconds:
+        b, h = int(rng.integers(w.B)), int(rng.integers(w.H))
+        rph = (rp[h * M:(h + 1) * M + 1] - rp[h * M]).astype(np.int32)
+        cih = ci[rp[h * M]:rp[(h + 1) * M]]
+        sl = (slice(b, b + 1), slice(h, h + 1))
+        t0 = time.perf_counter()
+        obw.backward(q[sl], k[sl], v[sl], do[sl], rph, cih, w.block_size, w.scale, w.causal)
+        elapsed += time.perf_counter() - t0
+        flops += 10.0 * w.block_size * w.block_size * w.d * len(cih)
+        done += 1
+    return flops / elapsed / 1e12, torch.get_num_threads(), done, elapsed
+
+
+def run_backward(args, w, rank, world, local_rank):
+    import torch
+
+    import block_sparse_attention_38_b200 as bsa
+
+    if w.pattern.kind == workloads.TOPK:
+        raise SystemExit("--backward runs on host-built patterns")
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    bsa.library()
+    q_h, k_h, v_h = workloads.make_qkv(w, seed=replica_seed(w, rank))
+    g = torch.Generator().manual_seed(replica_seed(w, rank) + 77)
+    do_h = torch.randn(q_h.shape, generator=g).to(torch.bfloat16)
+    q, k, v, do = (t.to(dev) for t in (q_h, k_h, v_h, do_h))
+    rp_np, ci_np = bsa.build_pattern_from(w.pattern)
+    cp_np, ri_np = bsa.transpose_pattern(rp_np, ci_np, w.H, w.M)
+    rp, ci, cp, ri = (torch.from_numpy(x).to(dev) for x in (rp_np, ci_np, cp_np, ri_np))
+    O, L = bsa.forward(q, k, v, rp, ci, w.block_size, w.scale, w.causal)
+    ws = torch.empty(w.B * w.H * w.N, dtype=torch.float32, device=dev)
+    flops = backward_flops(w, len(ci_np))
+    flush = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        return bsa.backward(q, k, v, O, do, L, rp, ci, cp, ri, w.block_size, w.scale, w.causal,
+                            workspace=ws)
+
+    for _ in range(args.warmup):
+        flush.fill_(1)
+        step()
+    torch.cuda.synchronize()
+    bsa.backward_status(clear=True)
+    visible = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+    ids = [x.strip() for x in visible.split(",") if x.strip()]
+    clocks = ClockSampler(ids[local_rank] if local_rank < len(ids) else str(local_rank))
+    if rank == 0:
+        clocks.start()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush.fill_(i & 0xFF)
+        starts[i].record(stream)
+        step()
+        ends[i].record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clock_info = clocks.stop() if rank == 0 else None
+    per_step = [s_.elapsed_time(e) for s_, e in zip(starts, ends)]
+    total_ms = float(sum(per_step))
+    if bsa.backward_status(clear=True) or bsa.device_status(clear=True):
+        raise RuntimeError("backward kernels reported a device status")
+
+    # End to end through the public API: Q, K, V, O, dO, LSE and the two CSR
+    # copies from pinned host memory, the backward, dQ, dK, dV back to pinned
+    # host memory, every step.
+    hosts = [t.cpu().pin_memory() for t in (q, k, v, O, do, L)]
+    hcsr = [torch.from_numpy(x).pin_memory() for x in (rp_np, ci_np, cp_np, ri_np)]
+    devs = [torch.empty_like(t, device=dev) for t in hosts + hcsr]
+    outs_h = [torch.empty(q.shape, dtype=torch.bfloat16).pin_memory() for _ in range(3)]
+    h2d = sum(t.numel() * t.element_size() for t in hosts + hcsr)
+    d2h = sum(t.numel() * t.element_size() for t in outs_h)
+
+    def e2e_step():
+        for dst, src in zip(devs, hosts + hcsr):
+            dst.copy_(src, non_blocking=True)
+        grads = bsa.backward(*devs[:6], *devs[6:], w.block_size, w.scale, w.causal, workspace=ws)
+        for dst, src in zip(outs_h, grads):
+            dst.copy_(src, non_blocking=True)
+        return grads
+
+    for _ in range(max(1, args.warmup)):
+        e2e_step()
+    torch.cuda.synchronize()
+    e_steps = max(3, min(args.steps, 20))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(e_steps):
+        grads = e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / e_steps
+    if not all(torch.equal(hh, gg.cpu()) for hh, gg in zip(outs_h, grads)):
+        raise RuntimeError("end-to-end result differs from the device result")
+
+    total_ms, e2e_ms = max_over_ranks([total_ms, e2e_ms], world, device=dev)
+    if rank != 0:
+        return
+    ms = total_ms / args.steps
+    peaks, peak_src = load_peaks()
+    peak_tc = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    roof = {"bound": "tensor", "achieved": flops / (ms * 1e-3) / 1e12, "peak": peak_tc,
+            "unit": "TFLOP/s"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    tr = NCU_TRAFFIC.get(w.name + ":backward")
+    roof["traffic"] = tr[0] if tr and tr[1] == kernel_hash(BACKWARD_SOURCES) else None
+    roof["peak_source"] = f"{peak_src} (MEASURED_PEAKS.json burst)" if peak_src == "measured" else "fallback"
+    roof["kernel"] = "bsa::bwd::dot_kernel + dkdv_kernel + dq_kernel"
+    roof["kernel_ms"] = ms
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline and w.N > ORACLE_BACKWARD_MAX_N:
+        cpu = {"value": None, "unit": "TFLOP/s", "cores": 0, "kind": "oracle",
+               "sample": f"none: the dense fp64 backward oracle holds N x N arrays per (b, h), "
+                         f"too large at N = {w.N}"}
+    elif world == 1 and not args.no_cpu_baseline:
+        tf, threads, npairs, el = cpu_backward_sample(w, q_h, k_h, v_h, do_h, rp_np, ci_np,
+                                                      args.cpu_seconds)
+        cpu = {"value": tf, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+               "sample": f"{npairs} random (b, h) backward passes of {w.name} ({el:.1f} s, fp64)"}
+    line = {
+        "metric": METRIC, "value": whole_job_tflops(flops, world, ms), "unit": "TFLOP/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": w.name, "pass": "backward", "B": w.B, "H": w.H, "N": w.N,
+                   "d": w.d, "block_size": w.block_size, "nnz_blocks": int(len(ci_np)),
+                   "causal": bool(w.causal),
+                   "l2": "flushed before every timed step (512 MB write)",
+                   "parallelism": f"replicas x{world}"},
+        "roofline": roof,
+        "cpu_baseline": cpu,
+        "e2e": {"value": whole_job_tflops(flops, world, e2e_ms), "unit": "TFLOP/s",
+                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+                "ms_per_step": e2e_ms},
+        "gpu_launches": 3 * args.steps,
+        "clocks": clock_info,
+        "min_ms": min(per_step), "median_ms": statistics.median(per_step),
     }
     print(json.dumps(line), flush=True)
 
@@ -456,6 +638,44 @@ def run_decode(args, w, rank, world, local_rank):
         "gpu_launches": args.steps,
         "clocks": clock_info,
         "min_ms": min(per_step), "median_ms": statistics.median(per_step),
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_reference_backward(args, w, rank, world):
+    """fp64 CPU backward oracle on the host cores, each step a bounded sample of (b, h)."""
+    if rank != 0:
+        return
+    import torch
+
+    from oracle import patterns
+
+    if w.N > ORACLE_BACKWARD_MAX_N:
+        print(json.dumps({"impl": "reference", "unavailable":
+                          f"the dense fp64 backward oracle holds N x N arrays per (b, h), "
+                          f"too large at N = {w.N}"}), flush=True)
+        return
+    q, k, v = workloads.make_qkv(w)
+    g = torch.Generator().manual_seed(w.seed + 77)
+    do = torch.randn(q.shape, generator=g).to(torch.bfloat16)
+    rp, ci = patterns.csr(w.pattern)
+    vals, times, done, threads = [], [], 0, 0
+    for i in range(args.steps):
+        tf, threads, n, el = cpu_backward_sample(w, q, k, v, do, rp, ci, 2.0, rng_seed=i)
+        vals.append(tf)
+        times.append(el)
+        done += n
+    value = statistics.median(vals)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * statistics.mean(times), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "pass": "backward", "B": w.B, "H": w.H, "N": w.N,
+                   "d": w.d, "block_size": w.block_size},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                         "sample": f"{done} random (b, h) backward passes of {w.name} over {args.steps} steps"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
 
@@ -721,18 +941,22 @@ def main():
                     choices=list(workloads.WORKLOADS) + list(workloads.DECODE_WORKLOADS))
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--backward", action="store_true",
+                    help="time the backward pass (dQ, dK, dV) instead of the forward")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     decode = args.workload in workloads.DECODE_WORKLOADS
     w = (workloads.DECODE_WORKLOADS if decode else workloads.WORKLOADS)[args.workload]
-    run = run_decode if decode else run_ours
+    run = run_decode if decode else (run_backward if args.backward else run_ours)
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
-        (run_reference_decode if decode else run_reference)(args, w, rank, world)
+        ref = run_reference_decode if decode else (
+            run_reference_backward if args.backward else run_reference)
+        ref(args, w, rank, world)
         return
     if world > 1:
         import datetime
