@@ -20,10 +20,11 @@
 //                block rows' columns (the CSR), 128 keys a step:
 //                  S = Q K^T and dP = dO V^T; dS to TMEM; dQ += dS K.
 // Every output row is produced by exactly one CTA: no atomics, no scratch
-// beyond D.  The steps run one after another inside a CTA (TMA, MMA,
-// elementwise, MMA); tiles of different CTAs overlap.  Every wait is bounded;
-// a wait that gives up sets BSA_STATUS_TIMEOUT and the CTA finishes without
-// writing its tile.
+// beyond D.  Inside a CTA (8 warps: two per TMEM lane quadrant, one per half
+// of the 128 columns) a step runs its MMAs and its elementwise pass in turn
+// while the TMA gather of the next step is already in flight (two buffers).
+// Every wait is bounded; a wait that gives up sets BSA_STATUS_TIMEOUT and the
+// CTA finishes without writing its tile.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -41,7 +42,7 @@ namespace bwd {
 
 constexpr int kMaxM = 4096;
 constexpr int kWords = kMaxM / 32;
-constexpr int kThreads = 128;  // one thread per TMEM lane = tile row
+constexpr int kThreads = 256;  // two warps per TMEM lane quadrant: one per column half
 constexpr long long kWaitLimitCycles = 4000000000LL;  // ~2 s at 1.97 GHz
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -62,14 +63,14 @@ struct Cfg {
 
 struct Ctrl {
   uint64_t kv_bar;    // the CTA's own tile (K, V or Q, dO) landed
-  uint64_t ld_bar;    // the step's gathered tiles landed
+  uint64_t ld_bar[2]; // the gathered tiles of buffer 0 / 1 landed
   uint64_t mma_bar;   // the step's first two MMAs completed
   uint64_t mma2_bar;  // the step's accumulating MMAs completed
   uint64_t final_bar; // every MMA issued by the CTA completed (teardown)
   uint32_t tmem_base;
   volatile int abort;
   int n_steps;
-  int blk[4];                       // the step's blocks (-1: padding)
+  int blk[2][4];                    // each buffer's blocks (-1: padding)
   alignas(16) float lse2[128];      // dK/dV: the step's queries' LSE * log2(e)
   alignas(16) float dd[128];        // dK/dV: the step's queries' D
   uint32_t map[4][kWords];          // per tile block: the other side's blocks
@@ -240,13 +241,11 @@ __device__ __forceinline__ void next_blocks(const Ctrl* ctl, int W, int& w, uint
 
 __device__ __forceinline__ uint32_t pack2(float lo, float hi) { return pack_bf16x2(lo, hi); }
 
-// Writes rows [row0, row0 + 128) of a tile accumulator (D fp32 columns from
-// TMEM column `col`), times `mul`, as bf16 to out[bh, row0 + lane_row, :].
-template <int D>
-__device__ __forceinline__ void store_rows(uint32_t tmem_lane, int col, float mul,
-                                           __nv_bfloat16* out, long long row) {
-#pragma unroll
-  for (int g = 0; g < D / 32; ++g) {
+// Writes `groups` 32-column groups of this thread's accumulator row (fp32
+// TMEM columns from `col`), times `mul`, as bf16 to out[row, ocol..].
+__device__ __forceinline__ void store_groups(uint32_t tmem_lane, int col, int groups, float mul,
+                                             __nv_bfloat16* out, long long row, int D, int ocol) {
+  for (int g = 0; g < groups; ++g) {
     uint32_t r[32];
     tmem_ld32(tmem_lane + col + 32 * g, r);
     tmem_wait_ld();
@@ -256,18 +255,31 @@ __device__ __forceinline__ void store_rows(uint32_t tmem_lane, int col, float mu
 #pragma unroll
     for (int c = 0; c < 16; ++c)
       w[c] = pack2(__uint_as_float(r[2 * c]) * mul, __uint_as_float(r[2 * c + 1]) * mul);
-    uint4* dst = reinterpret_cast<uint4*>(out + row * D + 32 * g);
+    uint4* dst = reinterpret_cast<uint4*>(out + row * D + ocol + 32 * g);
 #pragma unroll
     for (int c = 0; c < 4; ++c) dst[c] = v[c];
   }
 }
 
-__device__ __forceinline__ void store_zero_rows(int D, __nv_bfloat16* out, long long row) {
-  uint4* dst = reinterpret_cast<uint4*>(out + row * D);
-  for (int c = 0; c < D / 8; ++c) dst[c] = make_uint4(0u, 0u, 0u, 0u);
+__device__ __forceinline__ void store_zero_cols(__nv_bfloat16* out, long long row, int D, int ocol,
+                                                int n) {
+  uint4* dst = reinterpret_cast<uint4*>(out + row * D + ocol);
+  for (int c = 0; c < n / 8; ++c) dst[c] = make_uint4(0u, 0u, 0u, 0u);
 }
 
+// Thread 0's view of the gathered-tile ring: two buffers, the k-th load of
+// buffer b completes phase k of ld_bar[b].
+struct Gather {
+  int uw = 0;
+  uint32_t ucur = 0;
+  int issued[2] = {0, 0};
+  int pending = 0;  // bit b: a load of buffer b not yet waited for
+};
+
 // ------------------------------------------------------------ dK, dV
+// Step s uses buffer s & 1; the gather of step s + 1 is issued as soon as
+// step s - 1's accumulating MMAs (the last readers of that buffer) are done,
+// so it lands while step s computes.
 template <int BS, int D>
 __global__ void __launch_bounds__(kThreads, 1)
     dkdv_kernel(const __grid_constant__ CUtensorMap tQ, const __grid_constant__ CUtensorMap tK,
@@ -279,11 +291,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   unsigned char* sK = smem;
   unsigned char* sV = smem + C::TILE;
-  unsigned char* sQ = smem + 2 * C::TILE;
-  unsigned char* sdO = smem + 3 * C::TILE;
-  Ctrl* ctl = reinterpret_cast<Ctrl*>(smem + 4 * C::TILE);
+  unsigned char* sQ = smem + 2 * C::TILE;   // two buffers
+  unsigned char* sdO = smem + 4 * C::TILE;  // two buffers
+  Ctrl* ctl = reinterpret_cast<Ctrl*>(smem + 6 * C::TILE);
 
-  const int tid = threadIdx.x, warp = tid >> 5;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int quad = warp & 3, half = warp >> 2;  // TMEM lane quadrant, column half
   const int tiles = a.N / 128;
   const int bh = static_cast<int>(blockIdx.x / tiles);
   const int kt = static_cast<int>(blockIdx.x % tiles);
@@ -297,7 +310,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   if (tid == 0) {
     mbar_init(&ctl->kv_bar, 1);
-    mbar_init(&ctl->ld_bar, 1);
+    mbar_init(&ctl->ld_bar[0], 1);
+    mbar_init(&ctl->ld_bar[1], 1);
     mbar_init(&ctl->mma_bar, 1);
     mbar_init(&ctl->mma2_bar, 1);
     mbar_init(&ctl->final_bar, 1);
@@ -309,43 +323,49 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = ctl->tmem_base;
-  const uint32_t tlane = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+  const uint32_t tlane = tmem + (static_cast<uint32_t>(quad * 32) << 16);
   const int steps = ctl->n_steps;
 
-  int uw = 0;
-  uint32_t ucur = ctl->uni[0];
-  bool loads_pending = false;  // thread 0: a gathered load not yet waited for
+  Gather gt;
+  gt.ucur = ctl->uni[0];
+  auto gather = [&](int st) {  // thread 0: the tiles of step st into buffer st & 1
+    const int b = st & 1;
+    int blk[4];
+    next_blocks(ctl, W, gt.uw, gt.ucur, C::R, blk);
+    for (int r = 0; r < C::R; ++r) ctl->blk[b][r] = blk[r];
+    mbar_arrive_expect_tx(&ctl->ld_bar[b], 2 * C::TILE);
+    load_blocks<BS, D>(sQ + b * C::TILE, &tQ, &ctl->ld_bar[b], blk, a.N, bh);
+    load_blocks<BS, D>(sdO + b * C::TILE, &tdO, &ctl->ld_bar[b], blk, a.N, bh);
+    ++gt.issued[b];
+    gt.pending |= 1 << b;
+  };
   if (tid == 0 && steps > 0) {
     int own[4];
     for (int r = 0; r < C::R; ++r) own[r] = kb0 + r;
     mbar_arrive_expect_tx(&ctl->kv_bar, 2 * C::TILE);
     load_blocks<BS, D>(sK, &tK, &ctl->kv_bar, own, a.N, bh);
     load_blocks<BS, D>(sV, &tV, &ctl->kv_bar, own, a.N, bh);
+    gather(0);
   }
 
-  const int k = tid;                        // key row of the tile
+  const int k = quad * 32 + lane;           // key row of the tile
   const int kb = k / BS;                    // its block within the tile
   const int ktok = kt * 128 + k;
   int done = 0;                             // steps whose accumulating MMAs were issued
   for (int s = 0; s < steps; ++s) {
+    const int b = s & 1;
     if (tid == 0) {
       if (s > 0 && !wait_bounded(&ctl->mma2_bar, (s - 1) & 1, &ctl->abort)) {
         // nothing more is issued; the teardown drains
-      } else {
-        int blk[4];
-        next_blocks(ctl, W, uw, ucur, C::R, blk);
-        for (int r = 0; r < C::R; ++r) ctl->blk[r] = blk[r];
-        mbar_arrive_expect_tx(&ctl->ld_bar, 2 * C::TILE);
-        load_blocks<BS, D>(sQ, &tQ, &ctl->ld_bar, blk, a.N, bh);
-        load_blocks<BS, D>(sdO, &tdO, &ctl->ld_bar, blk, a.N, bh);
-        loads_pending = true;
+      } else if (s + 1 < steps) {
+        gather(s + 1);
       }
     }
     __syncthreads();
     if (ctl->abort) break;
-    {
+    if (tid < 128) {
       const int r = tid / BS;
-      const int qb = ctl->blk[r];
+      const int qb = ctl->blk[b][r];
       if (qb >= 0) {
         const long long q = static_cast<long long>(bh) * a.N + qb * BS + tid % BS;
         ctl->lse2[tid] = a.LSE[q] * kLog2e;
@@ -357,12 +377,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (tid == 0) {
       bool ok = !(s == 0 && !wait_bounded(&ctl->kv_bar, 0, &ctl->abort));
-      ok = ok && wait_bounded(&ctl->ld_bar, s & 1, &ctl->abort);
+      ok = ok && wait_bounded(&ctl->ld_bar[b], (s >> 1) & 1, &ctl->abort);
       if (ok) {
-        loads_pending = false;
+        gt.pending &= ~(1 << b);
         tc_fence_after();
-        mma_ss<D>(tmem + C::TMEM_A, smem_u32(sK), smem_u32(sQ));   // S^T = K Q^T
-        mma_ss<D>(tmem + C::TMEM_B, smem_u32(sV), smem_u32(sdO));  // dP^T = V dO^T
+        mma_ss<D>(tmem + C::TMEM_A, smem_u32(sK), smem_u32(sQ + b * C::TILE));   // S^T = K Q^T
+        mma_ss<D>(tmem + C::TMEM_B, smem_u32(sV), smem_u32(sdO + b * C::TILE));  // dP^T = V dO^T
         umma_commit(&ctl->mma_bar);
       }
     }
@@ -371,16 +391,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (ctl->abort) break;
     tc_fence_after();
 
-    // this key row against the step's 128 queries, 32 at a time
+    // this key row against 64 of the step's 128 queries, 32 at a time
     bool member[4];
     int qb0[4];
 #pragma unroll
     for (int r = 0; r < C::R; ++r) {
-      qb0[r] = ctl->blk[r];
+      qb0[r] = ctl->blk[b][r];
       member[r] = qb0[r] >= 0 && ((ctl->map[kb][qb0[r] >> 5] >> (qb0[r] & 31)) & 1u);
     }
 #pragma unroll 1
-    for (int g = 0; g < 4; ++g) {
+    for (int gg = 0; gg < 2; ++gg) {
+      const int g = half * 2 + gg;
       uint32_t sr[32], dr[32];
       tmem_ld32(tlane + C::TMEM_A + 32 * g, sr);
       tmem_ld32(tlane + C::TMEM_B + 32 * g, dr);
@@ -417,8 +438,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     if (tid == 0) {
       tc_fence_after();
-      mma_ts<D>(tmem + C::TMEM_C, tmem + C::TMEM_A, smem_u32(sdO), s > 0);  // dV += P^T dO
-      mma_ts<D>(tmem + C::TMEM_D, tmem + C::TMEM_B, smem_u32(sQ), s > 0);   // dK += dS^T Q
+      mma_ts<D>(tmem + C::TMEM_C, tmem + C::TMEM_A, smem_u32(sdO + b * C::TILE), s > 0);  // dV
+      mma_ts<D>(tmem + C::TMEM_D, tmem + C::TMEM_B, smem_u32(sQ + b * C::TILE), s > 0);   // dK
       umma_commit(&ctl->mma2_bar);
     }
     done = s + 1;
@@ -429,19 +450,21 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (tid == 0) {
     umma_commit(&ctl->final_bar);  // arrives once every MMA issued so far has completed
     wait_drain(&ctl->final_bar, 0);
-    if (loads_pending) wait_drain(&ctl->ld_bar, done & 1);
+    for (int b = 0; b < 2; ++b)
+      if (gt.pending & (1 << b)) wait_drain(&ctl->ld_bar[b], (gt.issued[b] - 1) & 1);
     if (steps > 0) wait_drain(&ctl->kv_bar, 0);
   }
   __syncthreads();
   tc_fence_after();
   const long long row = static_cast<long long>(bh) * a.N + ktok;
   if (!ctl->abort) {
+    const int ocol = half * (D / 2);
     if (done == 0) {
-      store_zero_rows(D, a.out0, row);
-      store_zero_rows(D, a.out1, row);
+      store_zero_cols(a.out0, row, D, ocol, D / 2);
+      store_zero_cols(a.out1, row, D, ocol, D / 2);
     } else {
-      store_rows<D>(tlane, C::TMEM_C, 1.f, a.out0, row);
-      store_rows<D>(tlane, C::TMEM_D, a.scale, a.out1, row);
+      store_groups(tlane, C::TMEM_C + ocol, D / 64, 1.f, a.out0, row, D, ocol);
+      store_groups(tlane, C::TMEM_D + ocol, D / 64, a.scale, a.out1, row, D, ocol);
     }
   }
   tc_fence_before();
@@ -461,11 +484,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   unsigned char* sQ = smem;
   unsigned char* sdO = smem + C::TILE;
-  unsigned char* sK = smem + 2 * C::TILE;
-  unsigned char* sV = smem + 3 * C::TILE;
-  Ctrl* ctl = reinterpret_cast<Ctrl*>(smem + 4 * C::TILE);
+  unsigned char* sK = smem + 2 * C::TILE;  // two buffers
+  unsigned char* sV = smem + 4 * C::TILE;  // two buffers
+  Ctrl* ctl = reinterpret_cast<Ctrl*>(smem + 6 * C::TILE);
 
-  const int tid = threadIdx.x, warp = tid >> 5;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int quad = warp & 3, half = warp >> 2;
   const int tiles = a.N / 128;
   const int bh = static_cast<int>(blockIdx.x / tiles);
   const int qt = static_cast<int>(blockIdx.x % tiles);
@@ -479,7 +503,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   if (tid == 0) {
     mbar_init(&ctl->kv_bar, 1);
-    mbar_init(&ctl->ld_bar, 1);
+    mbar_init(&ctl->ld_bar[0], 1);
+    mbar_init(&ctl->ld_bar[1], 1);
     mbar_init(&ctl->mma_bar, 1);
     mbar_init(&ctl->mma2_bar, 1);
     mbar_init(&ctl->final_bar, 1);
@@ -491,50 +516,56 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = ctl->tmem_base;
-  const uint32_t tlane = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+  const uint32_t tlane = tmem + (static_cast<uint32_t>(quad * 32) << 16);
   const int steps = ctl->n_steps;
 
-  const int q = tid;                 // query row of the tile
+  const int q = quad * 32 + lane;    // query row of the tile
   const int rb = q / BS;             // its block row within the tile
   const int qtok = qt * 128 + q;
   const long long qrow = static_cast<long long>(bh) * a.N + qtok;
   const float lse2 = a.LSE[qrow] * kLog2e;
   const float dq_d = a.Dq[qrow];
 
-  int uw = 0;
-  uint32_t ucur = ctl->uni[0];
-  bool loads_pending = false;
+  Gather gt;
+  gt.ucur = ctl->uni[0];
+  auto gather = [&](int st) {
+    const int b = st & 1;
+    int blk[4];
+    next_blocks(ctl, W, gt.uw, gt.ucur, C::R, blk);
+    for (int r = 0; r < C::R; ++r) ctl->blk[b][r] = blk[r];
+    mbar_arrive_expect_tx(&ctl->ld_bar[b], 2 * C::TILE);
+    load_blocks<BS, D>(sK + b * C::TILE, &tK, &ctl->ld_bar[b], blk, a.N, bh);
+    load_blocks<BS, D>(sV + b * C::TILE, &tV, &ctl->ld_bar[b], blk, a.N, bh);
+    ++gt.issued[b];
+    gt.pending |= 1 << b;
+  };
   if (tid == 0 && steps > 0) {
     int own[4];
     for (int r = 0; r < C::R; ++r) own[r] = rb0 + r;
     mbar_arrive_expect_tx(&ctl->kv_bar, 2 * C::TILE);
     load_blocks<BS, D>(sQ, &tQ, &ctl->kv_bar, own, a.N, bh);
     load_blocks<BS, D>(sdO, &tdO, &ctl->kv_bar, own, a.N, bh);
+    gather(0);
   }
   int done = 0;
   for (int s = 0; s < steps; ++s) {
+    const int b = s & 1;
     if (tid == 0) {
       if (s > 0 && !wait_bounded(&ctl->mma2_bar, (s - 1) & 1, &ctl->abort)) {
-      } else {
-        int blk[4];
-        next_blocks(ctl, W, uw, ucur, C::R, blk);
-        for (int r = 0; r < C::R; ++r) ctl->blk[r] = blk[r];
-        mbar_arrive_expect_tx(&ctl->ld_bar, 2 * C::TILE);
-        load_blocks<BS, D>(sK, &tK, &ctl->ld_bar, blk, a.N, bh);
-        load_blocks<BS, D>(sV, &tV, &ctl->ld_bar, blk, a.N, bh);
-        loads_pending = true;
+      } else if (s + 1 < steps) {
+        gather(s + 1);
       }
     }
     __syncthreads();
     if (ctl->abort) break;
     if (tid == 0) {
       bool ok = !(s == 0 && !wait_bounded(&ctl->kv_bar, 0, &ctl->abort));
-      ok = ok && wait_bounded(&ctl->ld_bar, s & 1, &ctl->abort);
+      ok = ok && wait_bounded(&ctl->ld_bar[b], (s >> 1) & 1, &ctl->abort);
       if (ok) {
-        loads_pending = false;
+        gt.pending &= ~(1 << b);
         tc_fence_after();
-        mma_ss<D>(tmem + C::TMEM_A, smem_u32(sQ), smem_u32(sK));   // S = Q K^T
-        mma_ss<D>(tmem + C::TMEM_B, smem_u32(sdO), smem_u32(sV));  // dP = dO V^T
+        mma_ss<D>(tmem + C::TMEM_A, smem_u32(sQ), smem_u32(sK + b * C::TILE));   // S = Q K^T
+        mma_ss<D>(tmem + C::TMEM_B, smem_u32(sdO), smem_u32(sV + b * C::TILE));  // dP = dO V^T
         umma_commit(&ctl->mma_bar);
       }
     }
@@ -547,11 +578,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     int kb0[4];
 #pragma unroll
     for (int r = 0; r < C::R; ++r) {
-      kb0[r] = ctl->blk[r];
+      kb0[r] = ctl->blk[b][r];
       member[r] = kb0[r] >= 0 && ((ctl->map[rb][kb0[r] >> 5] >> (kb0[r] & 31)) & 1u);
     }
 #pragma unroll 1
-    for (int g = 0; g < 4; ++g) {
+    for (int gg = 0; gg < 2; ++gg) {
+      const int g = half * 2 + gg;
       uint32_t sr[32], dr[32];
       tmem_ld32(tlane + C::TMEM_A + 32 * g, sr);
       tmem_ld32(tlane + C::TMEM_B + 32 * g, dr);
@@ -583,25 +615,27 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     if (tid == 0) {
       tc_fence_after();
-      mma_ts<D>(tmem + C::TMEM_C, tmem + C::TMEM_A, smem_u32(sK), s > 0);  // dQ += dS K
+      mma_ts<D>(tmem + C::TMEM_C, tmem + C::TMEM_A, smem_u32(sK + b * C::TILE), s > 0);  // dQ += dS K
       umma_commit(&ctl->mma2_bar);
     }
     done = s + 1;
   }
 
   if (tid == 0) {
-    umma_commit(&ctl->final_bar);  // arrives once every MMA issued so far has completed
+    umma_commit(&ctl->final_bar);
     wait_drain(&ctl->final_bar, 0);
-    if (loads_pending) wait_drain(&ctl->ld_bar, done & 1);
+    for (int b = 0; b < 2; ++b)
+      if (gt.pending & (1 << b)) wait_drain(&ctl->ld_bar[b], (gt.issued[b] - 1) & 1);
     if (steps > 0) wait_drain(&ctl->kv_bar, 0);
   }
   __syncthreads();
   tc_fence_after();
   if (!ctl->abort) {
+    const int ocol = half * (D / 2);
     if (done == 0)
-      store_zero_rows(D, a.out0, qrow);
+      store_zero_cols(a.out0, qrow, D, ocol, D / 2);
     else
-      store_rows<D>(tlane, C::TMEM_C, a.scale, a.out0, qrow);
+      store_groups(tlane, C::TMEM_C + ocol, D / 64, a.scale, a.out0, qrow, D, ocol);
   }
   tc_fence_before();
   __syncthreads();
@@ -653,7 +687,7 @@ int launch(const void* Q, const void* K, const void* V, const void* dO, Args a, 
       !make_map(&tv, V, BH, a.N, D, BS) || !make_map(&tdo, dO, BH, a.N, D, BS))
     return BSA_ERR_CUDA;
   // At least ~120 KB, so that one CTA (and its 512 TMEM columns) owns each SM.
-  int smem = 4 * C::TILE + static_cast<int>(sizeof(Ctrl)) + 1024;
+  int smem = 6 * C::TILE + static_cast<int>(sizeof(Ctrl)) + 1024;
   if (smem < 120 * 1024) smem = 120 * 1024;
   if (cudaFuncSetAttribute(dkdv_kernel<BS, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            smem) != cudaSuccess ||
