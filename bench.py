@@ -60,8 +60,8 @@ NCU_TRAFFIC = {
     # the decode kernel, keyed by the hash of DECODE_SOURCES
     "decode_loglinear_32k": (175425792 + 3372544, "7be0c4ee875188a6"),
     # the backward's three kernels together (dot + dK/dV + dQ), one backward
-    "local_global_8k:backward": (134230272 + 3581696 + 340731392 + 115491072 + 333471744
-                                 + 55681792, "b99ddf4496188bae"),
+    "local_global_8k:backward": (134229248 + 4284160 + 336716800 + 111309568 + 330468096
+                                 + 55514880, "418be616a808a425"),
 }
 
 

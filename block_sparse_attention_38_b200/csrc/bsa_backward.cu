@@ -402,33 +402,45 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll 1
     for (int gg = 0; gg < 2; ++gg) {
       const int g = half * 2 + gg;
-      uint32_t sr[32], dr[32];
-      tmem_ld32(tlane + C::TMEM_A + 32 * g, sr);
-      tmem_ld32(tlane + C::TMEM_B + 32 * g, dr);
-      tmem_wait_ld();
-      reg_fence32(sr);
-      reg_fence32(dr);
-      uint32_t pp[16], dp[16];
-      // a 32-column group lies inside one block of the step (BS >= 32)
+      // A 32-column group lies inside one block of the step, and a warp's 32
+      // rows inside one block of the tile (BS >= 32): whether the pair is in
+      // the pattern is uniform over the warp.  Groups outside it only write
+      // zeros.
       const int rg = (32 * g) / BS;
       const bool mem_g = member[rg];
-      const int qtok0 = qb0[rg] * BS + (32 * g) % BS;
+      uint32_t pp[16], dp[16];
+      if (mem_g) {
+        uint32_t sr[32], dr[32];
+        tmem_ld32(tlane + C::TMEM_A + 32 * g, sr);
+        tmem_ld32(tlane + C::TMEM_B + 32 * g, dr);
+        tmem_wait_ld();
+        reg_fence32(sr);
+        reg_fence32(dr);
+        const int qtok0 = qb0[rg] * BS + (32 * g) % BS;
+        const float4* l4 = reinterpret_cast<const float4*>(ctl->lse2 + 32 * g);
+        const float4* d4 = reinterpret_cast<const float4*>(ctl->dd + 32 * g);
 #pragma unroll
-      for (int c = 0; c < 32; c += 2) {
-        float pv[2], dv[2];
+        for (int c = 0; c < 32; c += 4) {
+          const float4 lq = l4[c / 4], dq = d4[c / 4];
+          const float lv[4] = {lq.x, lq.y, lq.z, lq.w}, dvv[4] = {dq.x, dq.y, dq.z, dq.w};
+          float pv[4], dv[4];
 #pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int col = 32 * g + c + e;
-          const int qtok = qtok0 + c + e;
-          const bool allowed = mem_g && (!a.causal || qtok >= ktok);
-          const float p = allowed ? ex2_approx(__uint_as_float(sr[c + e]) * a.scale_log2 -
-                                               ctl->lse2[col])
-                                  : 0.f;
-          pv[e] = p;
-          dv[e] = p * (__uint_as_float(dr[c + e]) - ctl->dd[col]);
+          for (int e = 0; e < 4; ++e) {
+            const bool allowed = !a.causal || qtok0 + c + e >= ktok;
+            const float p = allowed ? ex2_approx(fmaf(__uint_as_float(sr[c + e]), a.scale_log2,
+                                                      -lv[e]))
+                                    : 0.f;
+            pv[e] = p;
+            dv[e] = p * (__uint_as_float(dr[c + e]) - dvv[e]);
+          }
+          pp[c / 2] = pack2(pv[0], pv[1]);
+          pp[c / 2 + 1] = pack2(pv[2], pv[3]);
+          dp[c / 2] = pack2(dv[0], dv[1]);
+          dp[c / 2 + 1] = pack2(dv[2], dv[3]);
         }
-        pp[c / 2] = pack2(pv[0], pv[1]);
-        dp[c / 2] = pack2(dv[0], dv[1]);
+      } else {
+#pragma unroll
+        for (int c = 0; c < 16; ++c) pp[c] = dp[c] = 0u;
       }
       tmem_st16(tlane + C::TMEM_A + 32 * g, pp);   // P^T over consumed S^T columns
       tmem_st16(tlane + C::TMEM_B + 32 * g, dp);   // dS^T over consumed dP^T columns
@@ -584,29 +596,34 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll 1
     for (int gg = 0; gg < 2; ++gg) {
       const int g = half * 2 + gg;
-      uint32_t sr[32], dr[32];
-      tmem_ld32(tlane + C::TMEM_A + 32 * g, sr);
-      tmem_ld32(tlane + C::TMEM_B + 32 * g, dr);
-      tmem_wait_ld();
-      reg_fence32(sr);
-      reg_fence32(dr);
-      uint32_t dp[16];
-      // a 32-column group lies inside one block of the step (BS >= 32)
+      // the pair (block row, key block of the group) is uniform over the warp
       const int rg = (32 * g) / BS;
       const bool mem_g = member[rg];
-      const int ktok0 = kb0[rg] * BS + (32 * g) % BS;
+      uint32_t dp[16];
+      if (mem_g) {
+        uint32_t sr[32], dr[32];
+        tmem_ld32(tlane + C::TMEM_A + 32 * g, sr);
+        tmem_ld32(tlane + C::TMEM_B + 32 * g, dr);
+        tmem_wait_ld();
+        reg_fence32(sr);
+        reg_fence32(dr);
+        const int ktok0 = kb0[rg] * BS + (32 * g) % BS;
 #pragma unroll
-      for (int c = 0; c < 32; c += 2) {
-        float dv[2];
+        for (int c = 0; c < 32; c += 2) {
+          float dv[2];
 #pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int ktok = ktok0 + c + e;
-          const bool allowed = mem_g && (!a.causal || ktok <= qtok);
-          const float p = allowed ? ex2_approx(__uint_as_float(sr[c + e]) * a.scale_log2 - lse2)
-                                  : 0.f;
-          dv[e] = p * (__uint_as_float(dr[c + e]) - dq_d);
+          for (int e = 0; e < 2; ++e) {
+            const bool allowed = !a.causal || ktok0 + c + e <= qtok;
+            const float p = allowed ? ex2_approx(fmaf(__uint_as_float(sr[c + e]), a.scale_log2,
+                                                      -lse2))
+                                    : 0.f;
+            dv[e] = p * (__uint_as_float(dr[c + e]) - dq_d);
+          }
+          dp[c / 2] = pack2(dv[0], dv[1]);
         }
-        dp[c / 2] = pack2(dv[0], dv[1]);
+      } else {
+#pragma unroll
+        for (int c = 0; c < 16; ++c) dp[c] = 0u;
       }
       tmem_st16(tlane + C::TMEM_A + 32 * g, dp);   // dS over consumed S columns
     }
