@@ -193,7 +193,31 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(rows)}
 
 
-def cpu_oracle_sample(w, q, k, v, rp, ci, seconds: float, rng_seed: int = 0):
+def cpu_model() -> str:
+    """The host CPU's model name (from /proc/cpuinfo), or '' when unknown."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return ""
+
+
+def causal_exact_flops(w, rp, ci) -> float:
+    """4 d flops per (query, key) pair the causal mask keeps: a stored block
+    j < i holds bs^2 pairs, the diagonal block bs (bs + 1) / 2."""
+    bs, M = w.block_size, w.M
+    pairs = 0
+    for h in range(w.H):
+        for i in range(M):
+            for j in ci[rp[h * M + i]:rp[h * M + i + 1]]:
+                pairs += bs * bs if j < i else (bs * (bs + 1) // 2 if j == i else 0)
+    return 4.0 * w.d * pairs * w.B
+
+
+def cpu_oracle_sample(w, q, k, v, rp, ci, seconds: float, rng_seed: int = 0, nthreads: int = 0):
     """Time the fp64 oracle on random query rows until `seconds` of work; returns
     (useful TFLOP/s, threads, rows done, seconds)."""
     import oracle
@@ -209,7 +233,7 @@ def cpu_oracle_sample(w, q, k, v, rp, ci, seconds: float, rng_seed: int = 0):
         r = (rows % w.N) // w.block_size
         t0 = time.perf_counter()
         _, _, threads = oracle.forward(q, k, v, rp, ci, w.block_size, w.scale, w.causal,
-                                       rows=rows)
+                                       rows=rows, nthreads=nthreads)
         elapsed += time.perf_counter() - t0
         flops += float((4.0 * w.block_size * w.d * lens[h * w.M + r]).sum())
         done_rows += batch
@@ -905,7 +929,13 @@ def run_ours(args, w, rank, world, local_rank):
         wo, qo, ko, vo, orp, oci = oracle_problem(w, q_h, k_h, v_h)
         tf, threads, nrows, el = cpu_oracle_sample(wo, qo, ko, vo, orp, oci, args.cpu_seconds)
         cpu = {"value": tf, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
-               "sample": f"{nrows} random query rows of {w.name} ({el:.1f} s, fp64)"}
+               "sample": f"{nrows} random query rows of {w.name} ({el:.1f} s, fp64)",
+               "nproc": os.cpu_count(), "cpu_model": cpu_model()}
+        if w.N <= 4096 and w.pattern.kind != workloads.TOPK:
+            # the same oracle on one thread, a shorter sample
+            tf1, _, n1, el1 = cpu_oracle_sample(wo, qo, ko, vo, orp, oci,
+                                                min(3.0, args.cpu_seconds), nthreads=1)
+            cpu["one_thread"] = {"value": tf1, "sample": f"{n1} random query rows ({el1:.1f} s)"}
 
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
@@ -924,6 +954,10 @@ def run_ours(args, w, rank, world, local_rank):
         "clocks": clock_info,
         "min_ms": min(per_step), "median_ms": statistics.median(per_step),
     }
+    if w.causal:
+        # the flops of the (query, key) pairs the causal mask keeps
+        line["causal_exact_tflops"] = whole_job_tflops(causal_exact_flops(w, rp_np, ci_np),
+                                                       world, ms)
     if topk:
         # the selection (block means + top-k select kernels) ahead of the forward
         line["config"]["top_k"] = w.pattern.top_k
