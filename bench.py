@@ -349,7 +349,8 @@ def run_backward(args, w, rank, world, local_rank):
     cp_np, ri_np = bsa.transpose_pattern(rp_np, ci_np, w.H, w.M)
     rp, ci, cp, ri = (torch.from_numpy(x).to(dev) for x in (rp_np, ci_np, cp_np, ri_np))
     O, L = bsa.forward(q, k, v, rp, ci, w.block_size, w.scale, w.causal)
-    ws = torch.empty(w.B * w.H * w.N, dtype=torch.float32, device=dev)
+    ws = torch.empty(int(bsa.library().bsa_backward_workspace_bytes(w.B, w.H, w.N)) // 4,
+                     dtype=torch.float32, device=dev)
     flops = backward_flops(w, len(ci_np))
     flush = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
@@ -436,7 +437,7 @@ def run_backward(args, w, rank, world, local_rank):
     tr = NCU_TRAFFIC.get(w.name + ":backward")
     roof["traffic"] = tr[0] if tr and tr[1] == kernel_hash(BACKWARD_SOURCES) else None
     roof["peak_source"] = f"{peak_src} (MEASURED_PEAKS.json burst)" if peak_src == "measured" else "fallback"
-    roof["kernel"] = "bsa::bwd::dot_kernel + dkdv_kernel + dq_kernel"
+    roof["kernel"] = "bsa::bwd::dot_kernel + tile_cost/order + dkdv_kernel + dq_kernel"
     roof["kernel_ms"] = ms
     cpu = None
     if world == 1 and not args.no_cpu_baseline and w.N > ORACLE_BACKWARD_MAX_N:
@@ -463,7 +464,7 @@ def run_backward(args, w, rank, world, local_rank):
         "e2e": {"value": whole_job_tflops(flops, world, e2e_ms), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                 "ms_per_step": e2e_ms},
-        "gpu_launches": 3 * args.steps,
+        "gpu_launches": 5 * args.steps,  # D, tile costs, tile orders, dK/dV, dQ
         "clocks": clock_info,
         "min_ms": min(per_step), "median_ms": statistics.median(per_step),
     }

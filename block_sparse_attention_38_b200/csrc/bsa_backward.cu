@@ -113,6 +113,7 @@ struct Args {
   const int32_t* idx;       // col_idx (dq) or row_idx (dkdv)
   __nv_bfloat16* out0;      // dQ (dq) or dV (dkdv)
   __nv_bfloat16* out1;      // dK (dkdv)
+  const int* order;         // tile processed by CTA x: order[x] (heaviest first)
   int H, N, M;
   float scale, scale_log2;
   int causal;
@@ -142,6 +143,69 @@ __global__ void dot_kernel(const __nv_bfloat16* __restrict__ O, const __nv_bfloa
     }
     for (int o = lanes_per_row / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
     if (r < rows && part == 0) Dq[r] = acc;
+  }
+}
+
+// --------------------------------------------------- heavy-first tile order
+// The cost of a tile is the total length of its R blocks' lists (an upper
+// bound of the union it walks).  Tiles whose blocks appear in long lists (a
+// global row or column) take many more steps than the rest; launched in
+// plain index order they would start late and leave a long tail, so the
+// tile kernels take their tiles heaviest first.
+constexpr int kCostBins = 4096;
+
+__global__ void tile_cost_kernel(const int32_t* __restrict__ ptr_a, const int32_t* __restrict__ ptr_b,
+                                 int H, int M, int R, int tiles_per_bh, long long T,
+                                 int* __restrict__ cost) {
+  const long long t = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (t >= T) return;
+  const long long bh = t / tiles_per_bh;
+  const int tile = static_cast<int>(t - bh * tiles_per_bh);
+  const long long base = static_cast<long long>(bh % H) * M + static_cast<long long>(tile) * R;
+  int ca = 0, cb = 0;
+  for (int r = 0; r < R; ++r) {
+    ca += max(0, ptr_a[base + r + 1] - ptr_a[base + r]);
+    cb += max(0, ptr_b[base + r + 1] - ptr_b[base + r]);
+  }
+  cost[t] = min(ca, kCostBins - 1);
+  cost[T + t] = min(cb, kCostBins - 1);
+}
+
+// Block x of the grid (x = 0, 1) orders the tiles of cost[x*T .. x*T+T) into
+// order[x*T ..]: by a counting sort on descending cost (ties in any order)
+// when the heaviest tile costs more than twice the mean, else in index order,
+// which keeps the tiles of one (b, h) together and their K/V shared in L2.
+__global__ void __launch_bounds__(1024) tile_order_kernel(const int* __restrict__ cost, long long T,
+                                                          int* __restrict__ order) {
+  __shared__ int hist[kCostBins];
+  __shared__ int sorted;
+  const int* c = cost + blockIdx.x * T;
+  int* o = order + blockIdx.x * T;
+  for (int b = threadIdx.x; b < kCostBins; b += blockDim.x) hist[b] = 0;
+  __syncthreads();
+  for (long long t = threadIdx.x; t < T; t += blockDim.x) atomicAdd(&hist[c[t]], 1);
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    long long total = 0;
+    int top = 0;
+    for (int b = 0; b < kCostBins; ++b) {
+      total += static_cast<long long>(b) * hist[b];
+      if (hist[b] > 0) top = b;
+    }
+    sorted = static_cast<long long>(top) * T > 2 * total;
+    int run = 0;  // exclusive offsets, heaviest bin first
+    for (int b = kCostBins - 1; b >= 0; --b) {
+      const int n = hist[b];
+      hist[b] = run;
+      run += n;
+    }
+  }
+  __syncthreads();
+  if (sorted) {
+    for (long long t = threadIdx.x; t < T; t += blockDim.x)
+      o[atomicAdd(&hist[c[t]], 1)] = static_cast<int>(t);
+  } else {
+    for (long long t = threadIdx.x; t < T; t += blockDim.x) o[t] = static_cast<int>(t);
   }
 }
 
@@ -298,8 +362,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int quad = warp & 3, half = warp >> 2;  // TMEM lane quadrant, column half
   const int tiles = a.N / 128;
-  const int bh = static_cast<int>(blockIdx.x / tiles);
-  const int kt = static_cast<int>(blockIdx.x % tiles);
+  const int tile_id = a.order[blockIdx.x];
+  const int bh = tile_id / tiles;
+  const int kt = tile_id % tiles;
   const int h = bh % a.H;
   const int kb0 = kt * C::R;
   const int W = (a.M + 31) / 32;
@@ -503,8 +568,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int quad = warp & 3, half = warp >> 2;
   const int tiles = a.N / 128;
-  const int bh = static_cast<int>(blockIdx.x / tiles);
-  const int qt = static_cast<int>(blockIdx.x % tiles);
+  const int tile_id = a.order[blockIdx.x];
+  const int bh = tile_id / tiles;
+  const int qt = tile_id % tiles;
   const int h = bh % a.H;
   const int rb0 = qt * C::R;
   const int W = (a.M + 31) / 32;
@@ -697,7 +763,8 @@ bool make_map(CUtensorMap* m, const void* base, long long BH, int N, int d, int 
 template <int BS, int D>
 int launch(const void* Q, const void* K, const void* V, const void* dO, Args a, long long BH,
            const int32_t* row_ptr, const int32_t* col_idx, const int32_t* col_ptr,
-           const int32_t* row_idx, void* dQ, void* dK, void* dV, cudaStream_t s) {
+           const int32_t* row_idx, void* dQ, void* dK, void* dV, int* cost, int* order,
+           cudaStream_t s) {
   using C = Cfg<BS, D>;
   CUtensorMap tq, tk, tv, tdo;
   if (!make_map(&tq, Q, BH, a.N, D, BS) || !make_map(&tk, K, BH, a.N, D, BS) ||
@@ -712,11 +779,19 @@ int launch(const void* Q, const void* K, const void* V, const void* dO, Args a, 
                            smem) != cudaSuccess)
     return BSA_ERR_CUDA;
   const unsigned grid = static_cast<unsigned>(BH * (a.N / 128));
+  const long long T = static_cast<long long>(grid);
+  // order[0..T): key tiles by their column lists; order[T..2T): query tiles by their rows
+  tile_cost_kernel<<<static_cast<unsigned>((T + 255) / 256), 256, 0, s>>>(
+      col_ptr, row_ptr, a.H, a.M, C::R, a.N / 128, T, cost);
+  if (cudaGetLastError() != cudaSuccess) return BSA_ERR_CUDA;
+  tile_order_kernel<<<2, 1024, 0, s>>>(cost, T, order);
+  if (cudaGetLastError() != cudaSuccess) return BSA_ERR_CUDA;
   Args kv = a;
   kv.ptr = col_ptr;
   kv.idx = row_idx;
   kv.out0 = static_cast<__nv_bfloat16*>(dV);
   kv.out1 = static_cast<__nv_bfloat16*>(dK);
+  kv.order = order;
   dkdv_kernel<BS, D><<<grid, kThreads, smem, s>>>(tq, tk, tv, tdo, kv);
   if (cudaGetLastError() != cudaSuccess) return BSA_ERR_CUDA;
   Args qa = a;
@@ -724,6 +799,7 @@ int launch(const void* Q, const void* K, const void* V, const void* dO, Args a, 
   qa.idx = col_idx;
   qa.out0 = static_cast<__nv_bfloat16*>(dQ);
   qa.out1 = nullptr;
+  qa.order = order + T;
   dq_kernel<BS, D><<<grid, kThreads, smem, s>>>(tq, tk, tv, tdo, qa);
   return cudaGetLastError() == cudaSuccess ? BSA_OK : BSA_ERR_CUDA;
 }
@@ -733,9 +809,13 @@ inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 }  // namespace bwd
 }  // namespace bsa
 
+// D (fp32 per query row), then the tile costs and the two tile orders (int
+// per 128-row tile, twice each).
 extern "C" size_t bsa_backward_workspace_bytes(int B, int H, int N) {
   if (B < 1 || H < 1 || N < 1) return 0;
-  return static_cast<size_t>(B) * static_cast<size_t>(H) * static_cast<size_t>(N) * sizeof(float);
+  const size_t rows = static_cast<size_t>(B) * static_cast<size_t>(H) * static_cast<size_t>(N);
+  const size_t tiles = static_cast<size_t>(B) * static_cast<size_t>(H) * ((N + 127) / 128);
+  return rows * sizeof(float) + 4 * tiles * sizeof(int);
 }
 
 extern "C" int bsa_backward(const void* Q, const void* K, const void* V, const void* O,
@@ -767,6 +847,8 @@ extern "C" int bsa_backward(const void* Q, const void* K, const void* V, const v
   if (workspace_bytes < bsa_backward_workspace_bytes(B, H, N)) return BSA_ERR_BUFFER_TOO_SMALL;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   float* Dq = static_cast<float*>(workspace);
+  int* cost = reinterpret_cast<int*>(Dq + BH * N);
+  int* order = cost + 2 * BH * (N / 128);
   const long long rows = BH * N;
   const int threads = 256;
   long long blocks = (rows * (d / 8) + threads - 1) / threads;
@@ -785,12 +867,12 @@ extern "C" int bsa_backward(const void* Q, const void* K, const void* V, const v
   a.causal = causal;
   const int key = block_size * 1000 + d;
   switch (key) {
-    case 32064: return launch<32, 64>(Q, K, V, dO, a, BH, row_ptr, col_idx, col_ptr, row_idx, dQ, dK, dV, s);
-    case 32128: return launch<32, 128>(Q, K, V, dO, a, BH, row_ptr, col_idx, col_ptr, row_idx, dQ, dK, dV, s);
-    case 64064: return launch<64, 64>(Q, K, V, dO, a, BH, row_ptr, col_idx, col_ptr, row_idx, dQ, dK, dV, s);
-    case 64128: return launch<64, 128>(Q, K, V, dO, a, BH, row_ptr, col_idx, col_ptr, row_idx, dQ, dK, dV, s);
-    case 128064: return launch<128, 64>(Q, K, V, dO, a, BH, row_ptr, col_idx, col_ptr, row_idx, dQ, dK, dV, s);
-    case 128128: return launch<128, 128>(Q, K, V, dO, a, BH, row_ptr, col_idx, col_ptr, row_idx, dQ, dK, dV, s);
+    case 32064: return launch<32, 64>(Q, K, V, dO, a, BH, row_ptr, col_idx, col_ptr, row_idx, dQ, dK, dV, cost, order, s);
+    case 32128: return launch<32, 128>(Q, K, V, dO, a, BH, row_ptr, col_idx, col_ptr, row_idx, dQ, dK, dV, cost, order, s);
+    case 64064: return launch<64, 64>(Q, K, V, dO, a, BH, row_ptr, col_idx, col_ptr, row_idx, dQ, dK, dV, cost, order, s);
+    case 64128: return launch<64, 128>(Q, K, V, dO, a, BH, row_ptr, col_idx, col_ptr, row_idx, dQ, dK, dV, cost, order, s);
+    case 128064: return launch<128, 64>(Q, K, V, dO, a, BH, row_ptr, col_idx, col_ptr, row_idx, dQ, dK, dV, cost, order, s);
+    case 128128: return launch<128, 128>(Q, K, V, dO, a, BH, row_ptr, col_idx, col_ptr, row_idx, dQ, dK, dV, cost, order, s);
     default: return BSA_ERR_UNSUPPORTED;
   }
 }

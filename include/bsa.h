@@ -249,8 +249,9 @@ int bsa_topk_pattern_static(const void* Q, const void* K, int BH, int N, int d, 
 int bsa_transpose_pattern(const int32_t* row_ptr, const int32_t* col_idx, int32_t H, int32_t M,
                           int32_t* col_ptr, int32_t* row_idx, int64_t cap, int64_t* nnz_out);
 
-/* Device workspace bytes bsa_backward needs (D = dO . O per query row, fp32):
- * 4 * B * H * N; 0 for invalid sizes. */
+/* Device workspace bytes bsa_backward needs: D = dO . O per query row (fp32),
+ * then per 128-row tile two costs and two positions of the heavy-first tile
+ * orders (int32): 4*B*H*N + 16*B*H*ceil(N/128); 0 for invalid sizes. */
 size_t bsa_backward_workspace_bytes(int B, int H, int N);
 
 /*
@@ -268,8 +269,10 @@ size_t bsa_backward_workspace_bytes(int B, int H, int N);
  * row_ptr / col_idx: the forward's block-CSR (device); col_ptr / row_idx: its
  * column-major copy from bsa_transpose_pattern (device).  dQ, dK, dV: device
  * bf16 [B, H, N, d], fully written.  workspace: device memory of at least
- * bsa_backward_workspace_bytes(B, H, N) bytes, 16-byte aligned (overwritten).
- * Enqueued on `stream` (three kernels); nothing allocated or synchronised.
+ * bsa_backward_workspace_bytes(B, H, N) bytes, 16-byte aligned (overwritten;
+ * nothing in it needs to start at zero).  Enqueued on `stream` (five kernels:
+ * D, the tile costs, the heavy-first tile orders, dK/dV, dQ); nothing
+ * allocated or synchronised.
  * Supported: d in {64, 128}; block_size in {32, 64, 128}; N % 128 == 0;
  * M <= 4096; 16-byte aligned tensors.  Else BSA_ERR_INVALID_ARG /
  * BSA_ERR_UNSUPPORTED with nothing launched; BSA_ERR_BUFFER_TOO_SMALL for a

@@ -88,5 +88,7 @@ def test_backward_unsupported(kw):
 
 
 def test_backward_short_workspace():
-    assert bsa.library().bsa_backward_workspace_bytes(1, 2, 512) == 4 * 2 * 512
-    assert _bwd(wsb=4 * 2 * 512 - 1) == bsa.ERR_BUFFER_TOO_SMALL
+    # D per query row (fp32), then two costs and two orders per 128-row tile (int32)
+    need = 4 * 2 * 512 + 4 * 4 * (2 * 512 // 128)
+    assert bsa.library().bsa_backward_workspace_bytes(1, 2, 512) == need
+    assert _bwd(wsb=need - 1) == bsa.ERR_BUFFER_TOO_SMALL
