@@ -173,9 +173,12 @@ __global__ void tile_cost_kernel(const int32_t* __restrict__ ptr_a, const int32_
 
 // Block x of the grid (x = 0, 1) orders the tiles of cost[x*T .. x*T+T) into
 // order[x*T ..]: by a counting sort on descending cost (ties in any order)
-// when the heaviest tile costs more than twice the mean, else in index order,
-// which keeps the tiles of one (b, h) together and their K/V shared in L2.
+// when the heaviest tile costs more than twice the mean, or when the launch
+// is a few waves (T < few_waves tiles) and the last, partial wave should hold
+// the lightest tiles; else in index order, which keeps the tiles of one
+// (b, h) together and their K/V shared in L2.
 __global__ void __launch_bounds__(1024) tile_order_kernel(const int* __restrict__ cost, long long T,
+                                                          long long few_waves,
                                                           int* __restrict__ order) {
   __shared__ int hist[kCostBins];
   __shared__ int sorted;
@@ -192,7 +195,7 @@ __global__ void __launch_bounds__(1024) tile_order_kernel(const int* __restrict_
       total += static_cast<long long>(b) * hist[b];
       if (hist[b] > 0) top = b;
     }
-    sorted = static_cast<long long>(top) * T > 2 * total;
+    sorted = static_cast<long long>(top) * T > 2 * total || T < few_waves;
     int run = 0;  // exclusive offsets, heaviest bin first
     for (int b = kCostBins - 1; b >= 0; --b) {
       const int n = hist[b];
@@ -784,7 +787,10 @@ int launch(const void* Q, const void* K, const void* V, const void* dO, Args a, 
   tile_cost_kernel<<<static_cast<unsigned>((T + 255) / 256), 256, 0, s>>>(
       col_ptr, row_ptr, a.H, a.M, C::R, a.N / 128, T, cost);
   if (cudaGetLastError() != cudaSuccess) return BSA_ERR_CUDA;
-  tile_order_kernel<<<2, 1024, 0, s>>>(cost, T, order);
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  tile_order_kernel<<<2, 1024, 0, s>>>(cost, T, 8LL * sms, order);
   if (cudaGetLastError() != cudaSuccess) return BSA_ERR_CUDA;
   Args kv = a;
   kv.ptr = col_ptr;
