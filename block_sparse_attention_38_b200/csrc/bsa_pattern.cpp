@@ -240,4 +240,4 @@ extern "C" int bsa_transpose_pattern(const int32_t* row_ptr, const int32_t* col_
   return BSA_OK;
 }
 
-extern "C" int bsa_version(void) { return 101; }
+extern "C" int bsa_version(void) { return 200; }  // 0.2.0: top-k, decode, backward

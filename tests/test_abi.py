@@ -40,11 +40,14 @@ def _declared_functions():
 def test_library_exports_every_declared_symbol():
     names = _declared_functions()
     assert {"bsa_build_pattern", "bsa_validate_pattern", "bsa_forward",
-            "bsa_device_status", "bsa_version"} <= set(names)
+            "bsa_device_status", "bsa_version", "bsa_topk_nnz", "bsa_topk_workspace_bytes",
+            "bsa_topk_pattern", "bsa_topk_pattern_static", "bsa_transpose_pattern",
+            "bsa_backward_workspace_bytes", "bsa_backward", "bsa_backward_status",
+            "bsa_decode", "bsa_decode_status"} <= set(names)
     lib = ctypes.CDLL(bsa.LIB_PATH)
     for n in names:
         assert hasattr(lib, n), n
-    assert bsa.version() >= 100
+    assert bsa.version() == 200
 
 
 def _cases():
