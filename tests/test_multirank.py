@@ -44,12 +44,14 @@ def _rank_main(rank, world, port, results):
         times = [1.0 + rank, 10.0 - 3 * rank, 0.5 * (rank + 1)]
         got = bench.max_over_ranks(times, world)
 
-        # replica inputs: same shapes, different seeds per rank
+        # replica inputs: same shapes, different seeds per rank (forward and decode)
         w = workloads.WORKLOADS["tiny_loglinear"]
         q, _, _ = workloads.make_qkv(w, seed=bench.replica_seed(w, rank))
-        checksum = float(q.float().sum())
-        sums = [0.0] * world
-        sums[rank] = checksum
+        wd = workloads.DECODE_WORKLOADS["decode_loglinear_4k"]
+        qd, _, _, _, _, lens = workloads.make_decode_inputs(wd, seed=bench.replica_seed(wd, rank))
+        sums = [0.0] * (2 * world)
+        sums[rank] = float(q.float().sum())
+        sums[world + rank] = float(qd.float().sum()) + float(lens.sum())
         t = torch.tensor(sums, dtype=torch.float64)
         dist.all_reduce(t)  # gather the checksums (sum of one-hot vectors)
 
@@ -88,6 +90,7 @@ def test_two_gloo_ranks_reduce_timings_and_keep_replicas_apart():
         got, sums, printed = res[r]
         assert got == pytest.approx(expect)
         assert sums[0] != sums[1]          # the two replicas hold different inputs
+        assert sums[2] != sums[3]          # ... and different decode batches
         assert printed == ""               # rank 1 does not print a reference line
 
 
