@@ -1,7 +1,9 @@
 /*
- * bsa.h -- C ABI of the B200 block-sparse attention forward.
+ * bsa.h -- C ABI of the B200 block-sparse attention library: the host
+ * pattern builder, the forward, and for the same patterns the backward pass,
+ * a decode step over a KV cache and content-based top-k block selection.
  *
- * The library computes O = softmax(scale * Q K^T) V in which every query
+ * The forward computes O = softmax(scale * Q K^T) V in which every query
  * row's softmax covers only the key blocks that its block row selects
  * ("Block Sparse Attention with Log-Linear Complexity", section 3.3: the
  * denominator sums only over the connected K blocks; unconnected positions
