@@ -10,12 +10,14 @@
 //
 // The work is a matrix-vector product streamed from HBM, so it runs on the
 // CUDA cores, fed by TMA:
-//   * one CTA per (b, h): a producer warp and kConsumerWarps consumer warps;
+//   * one CTA per (b, h): a producer warp and NW consumer warps (3 for
+//     d = 128, 4 for d = 64);
 //   * the producer dedups the CSR row into a bitmap of blocks j <= i, splits
 //     the blocks into units of 32 cache rows and TMA-loads each unit's K and
 //     V rows (128-byte swizzle) into shared-memory stages;
-//   * consumer warp w takes units w, w + kConsumerWarps, ... and owns the
-//     stages w, w + kConsumerWarps, ... (its own ring, used in order, so an
+//   * consumer warp w takes units w, w + NW, ... and owns the stages
+//     w, w + NW, ... (its own ring of 2 or 3 stages, used in order, so that
+//     the next unit's load overlaps the current unit's arithmetic, and so an
 //     mbarrier phase it waits for is never two phases ahead of the last one
 //     it consumed);
 //   * lane l scores key l of a unit (the swizzle makes the 32 row reads
@@ -42,8 +44,7 @@ namespace bsa {
 namespace decode {
 
 constexpr int kMaxM = 4096;
-constexpr int kConsumerWarps = 4;
-constexpr int kThreads = 32 * (kConsumerWarps + 1);
+constexpr int kMaxConsumerWarps = 4;
 constexpr int kStageBudget = 96 * 1024;
 constexpr long long kWaitLimitCycles = 4000000000LL;  // ~2 s at 1.97 GHz
 
@@ -57,15 +58,17 @@ struct Cfg {
   static constexpr int ATOM_BYTES = UK * 128;                   // one TMA box: 32 rows x 128 bytes
   static constexpr int HALF = ATOMS * ATOM_BYTES;               // the K (or the V) rows of a unit
   static constexpr int STAGE = 2 * HALF;                        // 8 KB (d = 64) or 16 KB (d = 128)
-  static constexpr int NSW = kStageBudget / (kConsumerWarps * STAGE);  // stages per consumer warp
-  static constexpr int NS = kConsumerWarps * NSW;               // 12 or 4 stages
+  static constexpr int NW = D == 128 ? 3 : 4;                   // consumer warps
+  static constexpr int THREADS = 32 * (NW + 1);                 // and one producer warp
+  static constexpr int NSW = kStageBudget / (NW * STAGE);       // stages per consumer warp: 3 or 2
+  static constexpr int NS = NW * NSW;                           // 12 or 6 stages
   static constexpr int CPL = D / 32;                            // output columns per lane
-  static_assert(NSW >= 1, "no stage per consumer warp");
+  static_assert(NSW >= 1 && NW <= kMaxConsumerWarps && NS <= 12, "stage ring");
   // unit u: consumer warp u % W, that warp's (u / W)-th unit
   __device__ static int stage(int u) {
-    return u % kConsumerWarps + kConsumerWarps * ((u / kConsumerWarps) % NSW);
+    return u % NW + NW * ((u / NW) % NSW);
   }
-  __device__ static uint32_t phase(int u) { return static_cast<uint32_t>(u / kConsumerWarps / NSW); }
+  __device__ static uint32_t phase(int u) { return static_cast<uint32_t>(u / NW / NSW); }
 };
 
 struct Ctrl {
@@ -76,9 +79,9 @@ struct Ctrl {
   int n_units;
   volatile int abort;
   alignas(16) float q[128];  // read as float4
-  float part_m[kConsumerWarps];
-  float part_l[kConsumerWarps];
-  float part_o[kConsumerWarps][128];
+  float part_m[kMaxConsumerWarps];
+  float part_l[kMaxConsumerWarps];
+  float part_o[kMaxConsumerWarps][128];
 };
 
 static_assert(offsetof(Ctrl, q) % 16 == 0, "q is read with 16-byte loads");
@@ -139,7 +142,7 @@ struct Args {
 };
 
 template <int D>
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__(Cfg<D>::THREADS, 2)
     decode_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
                   const Args a) {
   using C = Cfg<D>;
@@ -158,7 +161,7 @@ __global__ void __launch_bounds__(kThreads, 2)
   const int t = len_ok ? len - 1 : 0;
   const int i = t / a.bs;
 
-  if (warp == kConsumerWarps) {
+  if (warp == C::NW) {
     // ---------------------------------------------------------- producer setup
     if (lane == 0) {
       for (int s = 0; s < C::NS; ++s) {
@@ -213,13 +216,13 @@ __global__ void __launch_bounds__(kThreads, 2)
       ctl->n_units = (units - (diag ? 1 : 0)) * per_block + (diag ? last : 0);
     }
   } else {
-    for (int c = tid; c < D; c += kConsumerWarps * 32)
+    for (int c = tid; c < D; c += C::NW * 32)
       ctl->q[c] = __bfloat162float(a.q[bh * D + c]);
   }
   __syncthreads();
   const int n_units = ctl->n_units;
 
-  if (warp == kConsumerWarps) {
+  if (warp == C::NW) {
     // ------------------------------------------------------------- producer
     if (lane == 0) {
       int u = 0;
@@ -267,7 +270,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     for (int c = 0; c < C::CPL; ++c) o[c] = 0.f;
     const float4* q4 = reinterpret_cast<const float4*>(ctl->q);
 
-    for (int u = warp; u < n_units; u += kConsumerWarps) {
+    for (int u = warp; u < n_units; u += C::NW) {
       const int s = C::stage(u);
       const bool got = wait_bounded(&ctl->full[s], C::phase(u) & 1, &ctl->abort);
       if (!__all_sync(0xffffffffu, got)) break;
@@ -346,11 +349,11 @@ __global__ void __launch_bounds__(kThreads, 2)
   if (tid < D) {
     float mx = -INFINITY;
 #pragma unroll
-    for (int w = 0; w < kConsumerWarps; ++w) mx = fmaxf(mx, ctl->part_m[w]);
+    for (int w = 0; w < C::NW; ++w) mx = fmaxf(mx, ctl->part_m[w]);
     float out = 0.f, den = 0.f;
     if (mx != -INFINITY) {
 #pragma unroll
-      for (int w = 0; w < kConsumerWarps; ++w) {
+      for (int w = 0; w < C::NW; ++w) {
         const float f = ex2_approx(ctl->part_m[w] - mx);
         den += ctl->part_l[w] * f;
         out += ctl->part_o[w][tid] * f;
@@ -408,7 +411,7 @@ int launch(const Args& a, long long BH, const void* kc, const void* vc, cudaStre
   if (cudaFuncSetAttribute(decode_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            smem) != cudaSuccess)
     return BSA_ERR_CUDA;
-  decode_kernel<D><<<static_cast<unsigned>(BH), kThreads, smem, s>>>(tk, tv, a);
+  decode_kernel<D><<<static_cast<unsigned>(BH), C::THREADS, smem, s>>>(tk, tv, a);
   return cudaGetLastError() == cudaSuccess ? BSA_OK : BSA_ERR_CUDA;
 }
 
