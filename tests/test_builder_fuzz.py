@@ -1,6 +1,8 @@
-"""Property test of the host pattern builder (bsa_build_pattern): for random
-descriptors of every kind, the block-CSR equals the oracle's enumeration bit
-for bit (tests/test_abi.py holds the hand-picked cases)."""
+"""Property tests of the host-side integer work against the oracle, bit for
+bit: the pattern builder (bsa_build_pattern) on random descriptors of every
+kind, the column-major copy (bsa_transpose_pattern) on random CSRs with
+repeats and unsorted rows, and the closed-form top-k sizes (bsa_topk_nnz).
+tests/test_abi.py and tests/test_backward_abi.py hold the hand-picked cases."""
 import numpy as np
 from hypothesis import HealthCheck, given, settings
 from hypothesis import strategies as st
@@ -32,3 +34,34 @@ def test_builder_matches_oracle_on_random_descriptors(desc):
     assert np.array_equal(rp, orp)
     assert np.array_equal(ci, oci)
     assert bsa.validate_pattern(rp, ci, desc.H, desc.M, desc.causal) == bsa.OK
+
+
+@st.composite
+def csrs(draw):
+    H = draw(st.integers(1, 3))
+    M = draw(st.integers(1, 40))
+    rows = [draw(st.lists(st.integers(0, M - 1), max_size=8)) for _ in range(H * M)]
+    rp = np.zeros(H * M + 1, np.int32)
+    rp[1:] = np.cumsum([len(r) for r in rows])
+    ci = np.array([j for r in rows for j in r], np.int32)
+    return H, M, rp, ci
+
+
+@settings(max_examples=150, deadline=None)
+@given(csrs())
+def test_transpose_matches_oracle_on_random_csrs(case):
+    from oracle import backward as obw
+
+    H, M, rp, ci = case
+    cp, ri = bsa.transpose_pattern(rp, ci, H, M)
+    ocp, ori = obw.transpose_pattern(rp, ci, H, M)
+    assert np.array_equal(cp, ocp) and np.array_equal(ri, ori)
+
+
+@settings(max_examples=200, deadline=None)
+@given(st.integers(1, 64), st.integers(1, 4096), st.integers(0, 5000), st.booleans())
+def test_topk_nnz_closed_form_matches_the_row_lengths(BH, M, top_k, causal):
+    from oracle import topk
+
+    want = BH * sum(topk.row_length(i, M, top_k, causal) for i in range(M))
+    assert bsa.topk_nnz(BH, M, top_k, causal) == want
