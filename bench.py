@@ -117,7 +117,7 @@ def compulsory_bytes(w) -> float:
 
 
 # The files each kernel is compiled from (its .cu and what it includes).
-FORWARD_SOURCES = ("bsa_common.cuh", "bsa_forward.cu", "bsa_fwd_rows.cuh", "sm100_ptx.cuh")
+FORWARD_SOURCES = ("bsa_common.cuh", "bsa_forward.cu", "bsa_fwd_pp.cuh", "sm100_ptx.cuh")
 DECODE_SOURCES = ("bsa_decode.cu", "sm100_ptx.cuh")
 BACKWARD_SOURCES = ("bsa_backward.cu", "sm100_ptx.cuh")
 
@@ -921,7 +921,7 @@ def run_ours(args, w, rank, world, local_rank):
     roof["traffic"] = tr[0] if tr and tr[1] == kernel_hash() else None
     roof["peak_source"] = f"{peak_src} (MEASURED_PEAKS.json burst)" if peak_src == "measured" else "fallback"
     roof["roofline_frac_max_of_tc_hbm"] = max(t_tc, t_hbm) / (fwd_ms * 1e-3)
-    roof["kernel"] = "bsa::rows::fwd_kernel"
+    roof["kernel"] = "bsa::pp::fwd_kernel"
     roof["kernel_ms"] = fwd_ms
 
     # CPU baseline: the oracle, as it stands, on a bounded sample of rows.

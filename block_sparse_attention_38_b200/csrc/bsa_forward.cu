@@ -1,12 +1,13 @@
 // bsa_forward.cu -- host side of the block-sparse attention forward: argument
-// validation, TMA descriptor encoding and the launch of the sm_100a row-tile
-// kernel (one instantiation per block size and head dimension).  This file is
-// the library's only CUDA translation unit; the kernel lives in the headers it
-// includes.
+// validation, TMA descriptor encoding and the launch of the sm_100a two-slot
+// kernel (one instantiation per block size and head dimension), plus the
+// device status word.  The kernel lives in the headers this file includes;
+// the library's other CUDA translation units are bsa_topk.cu, bsa_decode.cu
+// and bsa_backward.cu.
 #include <mutex>
 
 #include "bsa_common.cuh"
-#include "bsa_fwd_rows.cuh"
+#include "bsa_fwd_pp.cuh"
 
 namespace bsa {
 
@@ -51,11 +52,15 @@ struct DeviceInfo {
   int sms = 0;
 };
 
-bool device_info(int dev, DeviceInfo* out) {
+std::mutex& device_mutex() {
   static std::mutex mu;
+  return mu;
+}
+
+bool device_info(int dev, DeviceInfo* out) {
   static DeviceInfo cache[64];
   if (dev < 0 || dev >= 64) return false;
-  std::lock_guard<std::mutex> lock(mu);
+  std::lock_guard<std::mutex> lock(device_mutex());
   DeviceInfo& di = cache[dev];
   if (di.sms == 0) {
     int sms = 0;
@@ -67,11 +72,26 @@ bool device_info(int dev, DeviceInfo* out) {
   return true;
 }
 
+// Raises the dynamic shared-memory limit of the <BS, D> kernel on `dev` to
+// `bytes` once per instantiation and device, under the device mutex.
 template <int BS, int D>
-int launch_rows(const void* Q, const void* K, const void* V, const int32_t* row_ptr,
-           const int32_t* col_idx, int B, int H, int N, float scale, int causal, void* O,
-           float* LSE, cudaStream_t stream) {
-  using C = rows::Cfg<BS, D>;
+bool ensure_smem_attr(int dev, int bytes) {
+  static int set_bytes[64] = {};
+  if (dev < 0 || dev >= 64) return false;
+  std::lock_guard<std::mutex> lock(device_mutex());
+  if (set_bytes[dev] >= bytes) return true;
+  if (cudaFuncSetAttribute(pp::fwd_kernel<BS, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           bytes) != cudaSuccess)
+    return false;
+  set_bytes[dev] = bytes;
+  return true;
+}
+
+template <int BS, int D>
+int launch_fwd(const void* Q, const void* K, const void* V, const int32_t* row_ptr,
+               const int32_t* col_idx, int B, int H, int N, float scale, int causal, void* O,
+               float* LSE, cudaStream_t stream) {
+  using C = pp::Cfg<BS, D>;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return BSA_ERR_CUDA;
   DeviceInfo di;
@@ -94,19 +114,13 @@ int launch_rows(const void* Q, const void* K, const void* V, const int32_t* row_
   a.num_tiles = BH * a.G;
   a.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
   a.causal = causal;
-  const int smem = C::OFF_CTRL + static_cast<int>(sizeof(rows::Ctrl)) + 1024;
-  // At least ~120 KB so that one CTA (and its 512 TMEM columns) owns each SM.
-  const int smem_req = smem < 120 * 1024 ? 120 * 1024 : smem;
-  static bool attr_set[64] = {};
-  if (!attr_set[dev]) {
-    if (cudaFuncSetAttribute(rows::fwd_kernel<BS, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             smem_req) != cudaSuccess)
-      return BSA_ERR_CUDA;
-    attr_set[dev] = true;
-  }
+  // stages, control block, the four tile-bitmap buffers, and 1024 bytes of alignment slack
+  const int smem = C::OFF_CTRL + static_cast<int>(sizeof(pp::Ctrl)) +
+                   4 * pp::bitmap_words<BS>(a.W) * 4 + 1024;
+  if (!ensure_smem_attr<BS, D>(dev, smem)) return BSA_ERR_CUDA;
   long long grid = a.num_tiles < di.sms ? a.num_tiles : di.sms;
-  if (grid > rows::kMaxGrid) grid = rows::kMaxGrid;
-  rows::fwd_kernel<BS, D><<<static_cast<unsigned>(grid), rows::kThreads, smem_req, stream>>>(tq, tk, tv, a);
+  if (grid > pp::kMaxGrid) grid = pp::kMaxGrid;
+  pp::fwd_kernel<BS, D><<<static_cast<unsigned>(grid), pp::kThreads, smem, stream>>>(tq, tk, tv, a);
   if (cudaGetLastError() != cudaSuccess) return BSA_ERR_CUDA;
   return BSA_OK;
 }
@@ -133,12 +147,12 @@ extern "C" int bsa_forward(const void* Q, const void* K, const void* V, const in
   if (static_cast<long long>(H) * (N / block_size) + 1 > 2147483647LL) return BSA_ERR_UNSUPPORTED;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   switch (block_size * 1000 + d) {
-    case 32064: return launch_rows<32, 64>(Q, K, V, row_ptr, col_idx, B, H, N, scale, causal, O, LSE, s);
-    case 32128: return launch_rows<32, 128>(Q, K, V, row_ptr, col_idx, B, H, N, scale, causal, O, LSE, s);
-    case 64064: return launch_rows<64, 64>(Q, K, V, row_ptr, col_idx, B, H, N, scale, causal, O, LSE, s);
-    case 64128: return launch_rows<64, 128>(Q, K, V, row_ptr, col_idx, B, H, N, scale, causal, O, LSE, s);
-    case 128064: return launch_rows<128, 64>(Q, K, V, row_ptr, col_idx, B, H, N, scale, causal, O, LSE, s);
-    case 128128: return launch_rows<128, 128>(Q, K, V, row_ptr, col_idx, B, H, N, scale, causal, O, LSE, s);
+    case 32064: return launch_fwd<32, 64>(Q, K, V, row_ptr, col_idx, B, H, N, scale, causal, O, LSE, s);
+    case 32128: return launch_fwd<32, 128>(Q, K, V, row_ptr, col_idx, B, H, N, scale, causal, O, LSE, s);
+    case 64064: return launch_fwd<64, 64>(Q, K, V, row_ptr, col_idx, B, H, N, scale, causal, O, LSE, s);
+    case 64128: return launch_fwd<64, 128>(Q, K, V, row_ptr, col_idx, B, H, N, scale, causal, O, LSE, s);
+    case 128064: return launch_fwd<128, 64>(Q, K, V, row_ptr, col_idx, B, H, N, scale, causal, O, LSE, s);
+    case 128128: return launch_fwd<128, 128>(Q, K, V, row_ptr, col_idx, B, H, N, scale, causal, O, LSE, s);
     default: return BSA_ERR_UNSUPPORTED;
   }
 }
