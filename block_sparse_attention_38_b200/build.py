@@ -2,8 +2,10 @@
 
     python -m block_sparse_attention_38_b200.build [--force] [--verbose-ptxas]
 
-The library holds the host pattern builder (bsa_pattern.cpp) and the forward
-launcher plus its kernels (bsa_forward.cu).  CUDA runtime is linked
+The library holds the host pattern builder (bsa_pattern.cpp) and four CUDA
+translation units: the forward launcher with its kernel (bsa_forward.cu),
+top-k block selection (bsa_topk.cu), the decode step (bsa_decode.cu) and
+the backward pass (bsa_backward.cu).  CUDA runtime is linked
 statically; the driver's tensor-map encoder is looked up at run time, so the
 library loads on a machine without a GPU (only compute calls need one).
 """

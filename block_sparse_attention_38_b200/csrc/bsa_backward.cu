@@ -268,10 +268,10 @@ __device__ void build_maps(Ctrl* ctl, const Args& a, int h, int kb0, int R, bool
   for (int r = 0; r < R; ++r) {
     const int own = kb0 + r;
     int e0 = a.ptr[static_cast<long long>(h) * a.M + own];
-    const int e1 = a.ptr[static_cast<long long>(h) * a.M + own + 1];
-    if (e1 < e0) {
+    int e1 = a.ptr[static_cast<long long>(h) * a.M + own + 1];
+    if (e0 < 0 || e1 < e0) {
       if (threadIdx.x == 0) atomicOr(&g_bwd_status, BSA_STATUS_BAD_ROW_PTR);
-      e0 = e1;
+      e0 = e1 = 0;
     }
     for (int e = e0 + static_cast<int>(threadIdx.x); e < e1; e += blockDim.x) {
       const int x = a.idx[e];

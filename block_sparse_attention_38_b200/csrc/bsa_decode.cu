@@ -190,9 +190,9 @@ __global__ void __launch_bounds__(Cfg<D>::THREADS, 2)
     if (len_ok) {
       rp0 = a.row_ptr[static_cast<long long>(h) * a.M + i];
       rp1 = a.row_ptr[static_cast<long long>(h) * a.M + i + 1];
-      if (rp1 < rp0) {
+      if (rp0 < 0 || rp1 < rp0) {
         if (lane == 0) atomicOr(&g_decode_status, BSA_STATUS_BAD_ROW_PTR);
-        rp1 = rp0;
+        rp0 = rp1 = 0;
       }
     }
     for (int e = rp0 + lane; e < rp1; e += 32) {

@@ -114,9 +114,9 @@ int launch_fwd(const void* Q, const void* K, const void* V, const int32_t* row_p
   a.num_tiles = BH * a.G;
   a.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
   a.causal = causal;
-  // stages, control block, the four tile-bitmap buffers, and 1024 bytes of alignment slack
+  // stages, control block, the tile-bitmap buffers, and 1024 bytes of alignment slack
   const int smem = C::OFF_CTRL + static_cast<int>(sizeof(pp::Ctrl)) +
-                   4 * pp::bitmap_words<BS>(a.W) * 4 + 1024;
+                   pp::kSlots * pp::kTiRing * pp::bitmap_words<BS>(a.W) * 4 + 1024;
   if (!ensure_smem_attr<BS, D>(dev, smem)) return BSA_ERR_CUDA;
   long long grid = a.num_tiles < di.sms ? a.num_tiles : di.sms;
   if (grid > pp::kMaxGrid) grid = pp::kMaxGrid;

@@ -15,20 +15,23 @@
 // neither loaded from TMEM nor exponentiated.
 //
 // One persistent CTA per SM holds two independent tile slots.  Each slot has
-// its own S and O in TMEM and its own softmax warpgroup, in which thread i
-// owns query row i of the tile (TMEM lane i): the row maximum and sum need
-// no exchange between threads.  The MMA warp alternates between the slots,
-// so the tensor core computes one slot's P V and next scores while the other
-// slot's warpgroup turns its scores into probabilities.  Roles (384 threads):
-//   warps 0-3   softmax and epilogue of slot 0
-//   warps 4-7   softmax and epilogue of slot 1
-//   warp 8      TMA loads of Q, K, V for both slots, in the MMA's order
-//   warp 9      tcgen05.mma issuer (and owner of the 512 TMEM columns)
-//   warps 10-11 tile builders of slot 0 / slot 1: take the slot's next tile
-//               from the schedule and turn its CSR rows into block bitmaps
+// its own S, P and O in TMEM, its own Q/K/V stages in shared memory, its own
+// producer warp and its own softmax warpgroup, in which thread i owns query
+// row i of the tile (TMEM lane i): the row maximum and sum need no exchange
+// between threads.  One MMA warp serves both slots without blocking on
+// either: it polls each slot's barriers and issues whichever slot's next
+// contraction is ready, so the tensor core works on one slot while the other
+// slot's warpgroup turns scores into probabilities.  Roles (384 threads):
+//   warps 0-3    softmax and epilogue of slot 0
+//   warps 4-7    softmax and epilogue of slot 1
+//   warps 8, 10  producer of slot 0 / slot 1: the slot's next tile from the
+//                schedule, its block bitmaps from the CSR rows, and the TMA
+//                loads of its Q, K, V (with an L2 prefetch of the next Q)
+//   warp 9       tcgen05.mma issuer (and owner of the 512 TMEM columns)
+//   warp 11      idle
 //
-// TMEM columns: S of slot s in [128 s, +128), P (bf16 pairs) over its first
-// 64 columns once the scores are in registers; O of slot s in [256 + d s, +d).
+// TMEM columns: S of slot s in [128 s, +128); P (bf16 pairs) over the first 64
+// columns of S (d = 128) or in [256 + 64 s, +64) (d = 64); O after them.
 //
 // Work split (`schedule`): the 2 * grid slots are scheduled as independent
 // workers.  Tiles whose estimated cost exceeds half of one slot's share are
@@ -45,15 +48,9 @@ namespace pp {
 constexpr int kSlots = 2;
 constexpr int kWarps = 12;
 constexpr int kThreads = 32 * kWarps;
-constexpr int kLoadWarp = 8;
+constexpr int kProdWarp = 8;                // producer of slot s is warp kProdWarp + 2 s
 constexpr int kMmaWarp = 9;
-constexpr int kBuildWarp = 10;              // builder of slot s is warp kBuildWarp + s
-constexpr int kLaunchRegs = 168;            // 65536 / kThreads, rounded down to a multiple of 8
-constexpr int kSoftRegs = 208;
-constexpr int kOtherRegs = 88;
-static_assert(4 * 32 * (kSlots * kSoftRegs + kOtherRegs) <= kThreads * kLaunchRegs,
-              "register split exceeds the launch's registers");
-static_assert(kThreads * kLaunchRegs <= 65536, "registers per SM");
+constexpr int kTiRing = 3;                  // tile-info entries per slot
 
 constexpr int kMaxGrid = 160;               // CTAs per launch (the host caps the grid)
 constexpr int kMaxVirt = kSlots * kMaxGrid; // slots scheduled as workers
@@ -69,17 +66,25 @@ struct Cfg {
   static constexpr int Q_BYTES = TM * D * 2;
   static constexpr int CH_BYTES = NK * D * 2;    // one K or V stage
   static constexpr int QB = D == 64 ? 2 : 1;     // Q buffers per slot
-  static constexpr int NKS = D == 64 ? 4 : 2;    // K stages (shared by both slots)
-  static constexpr int NVS = D == 64 ? 4 : 2;    // V stages
-  static constexpr int OFF_Q = 0;
-  static constexpr int OFF_K = kSlots * QB * Q_BYTES;
-  static constexpr int OFF_V = OFF_K + NKS * CH_BYTES;
-  static constexpr int OFF_CTRL = OFF_V + NVS * CH_BYTES;
+  static constexpr int KS = D == 64 ? 2 : 1;     // K stages per slot
+  static constexpr int VS = KS;                  // V stages per slot
+  static constexpr int SLOT_BYTES = QB * Q_BYTES + (KS + VS) * CH_BYTES;
+  __host__ __device__ static constexpr int off_q(int s) { return s * SLOT_BYTES; }
+  __host__ __device__ static constexpr int off_k(int s) { return s * SLOT_BYTES + QB * Q_BYTES; }
+  __host__ __device__ static constexpr int off_v(int s) { return off_k(s) + KS * CH_BYTES; }
+  static constexpr int OFF_CTRL = kSlots * SLOT_BYTES;
   static constexpr uint32_t TMEM_COLS = 512;
-  static constexpr uint32_t TMEM_O = 2 * 128;    // O of slot s at TMEM_O + D s
+  // For d = 64, P of a slot has 64 TMEM columns of its own, so the slot's
+  // next S can be computed while its P is still being written; for d = 128
+  // there is no room, and P is written over the first 64 columns of S.
+  static constexpr bool SEP_P = D == 64;
+  static constexpr uint32_t TMEM_P = SEP_P ? 2 * 128 : 0;
+  static constexpr uint32_t TMEM_O = SEP_P ? 2 * 128 + 2 * 64 : 2 * 128;  // O of slot s at TMEM_O + D s
+  __host__ __device__ static constexpr uint32_t p_col(int s) { return SEP_P ? TMEM_P + 64 * s : 128 * s; }
   static_assert((Q_BYTES % 1024) == 0 && (CH_BYTES % 1024) == 0, "1024-byte aligned stages");
   static_assert(TMEM_O + kSlots * D <= TMEM_COLS, "TMEM layout");
   static_assert(TM == NK, "Q and K tiles share one slice-offset formula");
+  static_assert(QB <= 2 && KS <= 2, "barrier arrays");
 };
 
 // The plan every CTA computes identically (see `schedule`).
@@ -92,7 +97,7 @@ struct Plan {
   int heavy_hg[kMaxHeavyGroups];    // heavy groups of one batch element, in order
 };
 
-// One slot's position in the plan (its builder warp advances it).
+// One slot's position in the plan (its producer warp advances it).
 struct Cursor {
   long long heavy[2];               // this slot's heavy tiles
   long long round;                  // next round of light tiles
@@ -107,13 +112,19 @@ struct TileInfo {
   int pad;
 };
 
+// The barriers of one slot.
+struct SlotBars {
+  uint64_t t_full[kTiRing], t_empty[kTiRing];  // tile-info ring
+  uint64_t q_full[2], q_empty[2];
+  uint64_t k_full[2], k_empty[2], v_full[2], v_empty[2];
+  uint64_t s_full, p_full, o_full;
+  uint64_t s_free, pv_done;                    // separate-P layout only
+};
+
 struct Ctrl {
-  uint64_t t_full[kSlots][2], t_empty[kSlots][2];
-  uint64_t q_full[kSlots][2], q_empty[kSlots][2];
-  uint64_t k_full[4], k_empty[4], v_full[4], v_empty[4];
-  uint64_t s_full[kSlots], p_full[kSlots], o_full[kSlots];
+  SlotBars sb[kSlots];
   uint64_t final_bar;
-  TileInfo info[kSlots][2];
+  TileInfo info[kSlots][kTiRing];
   Cursor cur[kSlots];
   uint32_t tmem_base;
   AbortFlag abort;
@@ -208,6 +219,7 @@ __device__ void schedule(const FwdArgs& a, Ctrl* ctl) {
   for (long long hg = lo; hg < hi && n_hv > 0; ++hg) {
     if (group_cost<BS>(a, hg) > thr) pl.heavy_hg[hexcl++] = static_cast<int>(hg);
   }
+  __syncthreads();  // every thread's heavy groups are written before thread 0 deals them out
   if (tid == 0) {
     const long long Kh = Kg * nb;  // < 2V <= kMaxHeavyGroups
     const long long n_light = a.num_tiles - Kh;
@@ -273,33 +285,59 @@ __device__ __forceinline__ long long next_tile(const FwdArgs& a, const Plan& pl,
   return t;
 }
 
-// ------------------------------------------------------------- tile builder
-// Warp kBuildWarp + s: for each tile of slot s, the R block-row bitmaps and
-// their union from the CSR rows, published in the slot's two-entry ring.
+// ---------------------------------------------------------- producer warps
+// Warp kProdWarp + 2s, for slot s: take the slot's next tile from the
+// schedule, turn its CSR rows into the R block-row bitmaps and their union
+// (all lanes), publish it in the slot's tile-info ring, and issue (lane 0)
+// the TMA loads of its Q and, step by step, K and V into the slot's stages.
+// The tile after it is looked up at the same time and its Q prefetched into L2.
 template <int BS, int D>
-__device__ void build_role(int s, const FwdArgs& a, Ctrl* ctl, uint32_t* bitmaps) {
+__device__ void produce_role(int s, const CUtensorMap* tmQ, const CUtensorMap* tmK,
+                             const CUtensorMap* tmV, const FwdArgs& a, uint8_t* smem, Ctrl* ctl,
+                             uint32_t* bitmaps) {
   using C = Cfg<BS, D>;
   const int lane = threadIdx.x & 31;
   const int W = a.W;
   const int BMW = bitmap_words<BS>(W);
   const long long v = static_cast<long long>(kSlots) * blockIdx.x + s;
+  SlotBars& B = ctl->sb[s];
+  uint32_t q_loads = 0, k_loads = 0, v_loads = 0;
+  long long peeked = -2;  // lane 0: the slot's next tile, once looked up
+  bool ok = true;
+  if (lane == 0) {
+    prefetch_tensormap(tmQ);
+    prefetch_tensormap(tmK);
+    prefetch_tensormap(tmV);
+  }
   for (int t = 0;; ++t) {
-    const int buf = t & 1;
+    const int buf = t % kTiRing;
     int w_ok = 1;
     long long tile = -1;
     if (lane == 0) {
-      w_ok = wait_bounded(&ctl->t_empty[s][buf], ((t >> 1) & 1) ^ 1, &ctl->abort);
-      if (w_ok) tile = next_tile(a, ctl->plan, ctl->cur[s], v);
+      w_ok = wait_bounded(&B.t_empty[buf], ((t / kTiRing) & 1) ^ 1, &ctl->abort);
+      if (w_ok) {
+        tile = peeked == -2 ? next_tile(a, ctl->plan, ctl->cur[s], v) : peeked;
+        peeked = tile >= 0 ? next_tile(a, ctl->plan, ctl->cur[s], v) : -1;
+        if (peeked >= 0) {  // the next tile's Q into L2
+          const long long pbh = peeked / a.G;
+          const int pg = static_cast<int>(peeked - pbh * a.G);
+#pragma unroll
+          for (int ka = 0; ka < C::KATOMS; ++ka)
+            tma_prefetch_3d(tmQ, ka * 64, pg * C::TM, static_cast<int>(pbh));
+        }
+      }
     }
-    if (!__shfl_sync(0xffffffffu, w_ok, 0)) return;
+    if (!__shfl_sync(0xffffffffu, w_ok, 0)) { ok = false; break; }
     tile = __shfl_sync(0xffffffffu, tile, 0);
-    uint32_t* bm = bitmaps + (s * 2 + buf) * BMW;
+    uint32_t* bm = bitmaps + (s * kTiRing + buf) * BMW;
     int n = 0;
+    long long bh = 0;
+    int g = 0;
     if (tile >= 0) {
       for (int w = lane; w < BMW; w += 32) bm[w] = 0u;
       __syncwarp();
-      const long long bh = tile / a.G;
-      const int g = static_cast<int>(tile - bh * a.G);
+      bh = tile / a.G;
+      g = static_cast<int>(tile - bh * a.G);
       const int h = static_cast<int>(bh % a.H);
       for (int i = 0; i < C::R; ++i) {
         const int r = g * C::R + i;
@@ -330,255 +368,205 @@ __device__ void build_role(int s, const FwdArgs& a, Ctrl* ctl, uint32_t* bitmaps
       ctl->info[s][buf].n = n;
     }
     __syncwarp();
-    if (lane == 0) mbar_arrive(&ctl->t_full[s][buf]);
-    if (tile < 0) return;
-  }
-}
-
-// ------------------------------------------------------------ producer warp
-// Lane 0 issues every TMA load in the order the MMA issuer consumes them:
-// K(0) of each slot, then per slot in turn V(j) and the slot's next K (the
-// next step of its tile, or step 0 of its next tile after that tile's Q).
-template <int BS, int D>
-__device__ void load_role(const CUtensorMap* tmQ, const CUtensorMap* tmK, const CUtensorMap* tmV,
-                          const FwdArgs& a, uint8_t* smem, Ctrl* ctl, const uint32_t* bitmaps) {
-  using C = Cfg<BS, D>;
-  if ((threadIdx.x & 31) != 0) return;
-  prefetch_tensormap(tmQ);
-  prefetch_tensormap(tmK);
-  prefetch_tensormap(tmV);
-  const int W = a.W;
-  const int BMW = bitmap_words<BS>(W);
-  uint32_t q_loads[kSlots] = {0, 0}, k_loads = 0, v_loads = 0;
-  int t[kSlots] = {0, 0}, steps[kSlots] = {0, 0}, j[kSlots] = {0, 0};
-  bool active[kSlots] = {true, true};
-  long long bh[kSlots] = {0, 0};
-  int row0[kSlots][C::BPS];
-  // union bitmap walk of each slot's current tile
-  const uint32_t* ubits[kSlots] = {nullptr, nullptr};
-  int uw[kSlots] = {0, 0};
-  uint32_t ucur[kSlots] = {0, 0};
-  bool ok = true;
-
-  auto next_block = [&](int s) -> int {
-    while (ucur[s] == 0) {
-      if (++uw[s] >= W) return -1;
-      ucur[s] = ubits[s][uw[s]];
-    }
-    const int b = __ffs(ucur[s]) - 1;
-    ucur[s] &= ucur[s] - 1;
-    return uw[s] * 32 + b;
-  };
-  // Moves slot s to its next non-empty tile and loads that tile's Q.
-  auto next_tile_of = [&](int s) -> bool {
-    for (;;) {
-      const int buf = t[s] & 1;
-      if (!wait_bounded(&ctl->t_full[s][buf], (t[s] >> 1) & 1, &ctl->abort)) return false;
-      const long long tile = ctl->info[s][buf].tile;
-      const int n = ctl->info[s][buf].n;
-      if (tile < 0) {
-        active[s] = false;
-        return true;
+    if (lane == 0) mbar_arrive(&B.t_full[buf]);
+    if (tile < 0) break;
+    if (lane == 0) {
+      if (n > 0) {
+        const uint32_t qb = q_loads % C::QB;
+        ok = wait_bounded(&B.q_empty[qb], ((q_loads / C::QB) & 1) ^ 1, &ctl->abort);
+        if (ok) {
+          mbar_arrive_expect_tx(&B.q_full[qb], C::Q_BYTES);
+#pragma unroll
+          for (int ka = 0; ka < C::KATOMS; ++ka)
+            tma_load_3d(smem + C::off_q(s) + qb * C::Q_BYTES + ka * (C::TM * 128), tmQ, &B.q_full[qb],
+                        ka * 64, g * C::TM, static_cast<int>(bh));
+          ++q_loads;
+        }
+        BitIter it(bm + C::R * W, W);
+        const int steps = (n + C::BPS - 1) / C::BPS;
+        for (int j = 0; ok && j < steps; ++j) {
+          int row0[C::BPS];  // first token of each block of the step; N (out of range) pads
+#pragma unroll
+          for (int b = 0; b < C::BPS; ++b) {
+            const int jb = it.next();
+            row0[b] = jb >= 0 ? jb * BS : a.N;
+          }
+          const uint32_t ks = k_loads % C::KS;
+          ok = wait_bounded(&B.k_empty[ks], ((k_loads / C::KS) & 1) ^ 1, &ctl->abort);
+          if (!ok) break;
+          mbar_arrive_expect_tx(&B.k_full[ks], C::CH_BYTES);
+#pragma unroll
+          for (int b = 0; b < C::BPS; ++b)
+#pragma unroll
+            for (int ka = 0; ka < C::KATOMS; ++ka)
+              tma_load_3d(smem + C::off_k(s) + ks * C::CH_BYTES + ka * (C::NK * 128) + b * (BS * 128),
+                          tmK, &B.k_full[ks], ka * 64, row0[b], static_cast<int>(bh));
+          ++k_loads;
+          const uint32_t vs = v_loads % C::VS;
+          ok = wait_bounded(&B.v_empty[vs], ((v_loads / C::VS) & 1) ^ 1, &ctl->abort);
+          if (!ok) break;
+          mbar_arrive_expect_tx(&B.v_full[vs], C::CH_BYTES);
+#pragma unroll
+          for (int b = 0; b < C::BPS; ++b)
+#pragma unroll
+            for (int ka = 0; ka < C::KATOMS; ++ka)
+              tma_load_3d(smem + C::off_v(s) + vs * C::CH_BYTES + ka * (C::NK * 128) + b * (BS * 128),
+                          tmV, &B.v_full[vs], ka * 64, row0[b], static_cast<int>(bh));
+          ++v_loads;
+        }
       }
-      if (n == 0) {
-        mbar_arrive(&ctl->t_empty[s][buf]);
-        ++t[s];
-        continue;
-      }
-      bh[s] = tile / a.G;
-      const int g = static_cast<int>(tile - bh[s] * a.G);
-      ubits[s] = bitmaps + (s * 2 + buf) * BMW + C::R * W;
-      uw[s] = 0;
-      ucur[s] = ubits[s][0];
-      steps[s] = (n + C::BPS - 1) / C::BPS;
-      j[s] = 0;
-      const uint32_t qb = q_loads[s] % C::QB;
-      if (!wait_bounded(&ctl->q_empty[s][qb], ((q_loads[s] / C::QB) & 1) ^ 1, &ctl->abort))
-        return false;
-      mbar_arrive_expect_tx(&ctl->q_full[s][qb], C::Q_BYTES);
-      uint8_t* qdst = smem + C::OFF_Q + (s * C::QB + qb) * C::Q_BYTES;
-#pragma unroll
-      for (int ka = 0; ka < C::KATOMS; ++ka)
-        tma_load_3d(qdst + ka * (C::TM * 128), tmQ, &ctl->q_full[s][qb], ka * 64, g * C::TM,
-                    static_cast<int>(bh[s]));
-      ++q_loads[s];
-      return true;
+      if (ok) mbar_arrive(&B.t_empty[buf]);  // the producer is done with this tile's bitmaps
     }
-  };
-  auto issue_k = [&](int s) -> bool {
-#pragma unroll
-    for (int b = 0; b < C::BPS; ++b) {
-      const int jb = next_block(s);
-      row0[s][b] = jb >= 0 ? jb * BS : a.N;  // N (out of range) pads with zeros
-    }
-    const uint32_t ks = k_loads % C::NKS;
-    if (!wait_bounded(&ctl->k_empty[ks], ((k_loads / C::NKS) & 1) ^ 1, &ctl->abort)) return false;
-    mbar_arrive_expect_tx(&ctl->k_full[ks], C::CH_BYTES);
-#pragma unroll
-    for (int b = 0; b < C::BPS; ++b)
-#pragma unroll
-      for (int ka = 0; ka < C::KATOMS; ++ka)
-        tma_load_3d(smem + C::OFF_K + ks * C::CH_BYTES + ka * (C::NK * 128) + b * (BS * 128), tmK,
-                    &ctl->k_full[ks], ka * 64, row0[s][b], static_cast<int>(bh[s]));
-    ++k_loads;
-    return true;
-  };
-  auto issue_v = [&](int s) -> bool {
-    const uint32_t vs = v_loads % C::NVS;
-    if (!wait_bounded(&ctl->v_empty[vs], ((v_loads / C::NVS) & 1) ^ 1, &ctl->abort)) return false;
-    mbar_arrive_expect_tx(&ctl->v_full[vs], C::CH_BYTES);
-#pragma unroll
-    for (int b = 0; b < C::BPS; ++b)
-#pragma unroll
-      for (int ka = 0; ka < C::KATOMS; ++ka)
-        tma_load_3d(smem + C::OFF_V + vs * C::CH_BYTES + ka * (C::NK * 128) + b * (BS * 128), tmV,
-                    &ctl->v_full[vs], ka * 64, row0[s][b], static_cast<int>(bh[s]));
-    ++v_loads;
-    return true;
-  };
-
-  for (int s = 0; ok && s < kSlots; ++s) {
-    ok = next_tile_of(s);
-    if (ok && active[s]) ok = issue_k(s);
+    if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) { ok = false; break; }
   }
-  while (ok && (active[0] || active[1])) {
-    for (int s = 0; ok && s < kSlots; ++s) {
-      if (!active[s]) continue;
-      ok = issue_v(s);
-      if (!ok) break;
-      if (j[s] == steps[s] - 1) {
-        mbar_arrive(&ctl->t_empty[s][t[s] & 1]);
-        ++t[s];
-        ok = next_tile_of(s);
-        if (ok && active[s]) ok = issue_k(s);
-      } else {
-        ++j[s];
-        ok = issue_k(s);
-      }
-    }
-  }
-  if (ok) return;
+  if (ok || lane != 0) return;
   // On an early exit, let every copy already issued land before the CTA ends.
-  for (int s = 0; s < kSlots; ++s)
-    for (uint32_t b = 0; b < static_cast<uint32_t>(C::QB); ++b)
-      if (q_loads[s] > b) {
-        const uint32_t last = b + C::QB * ((q_loads[s] - 1 - b) / C::QB);
-        wait_drain(&ctl->q_full[s][b], (last / C::QB) & 1);
-      }
-  for (uint32_t st = 0; st < static_cast<uint32_t>(C::NKS); ++st)
-    if (k_loads > st) {
-      const uint32_t last = st + C::NKS * ((k_loads - 1 - st) / C::NKS);
-      wait_drain(&ctl->k_full[st], (last / C::NKS) & 1);
+  for (uint32_t b = 0; b < static_cast<uint32_t>(C::QB); ++b)
+    if (q_loads > b) {
+      const uint32_t last = b + C::QB * ((q_loads - 1 - b) / C::QB);
+      wait_drain(&B.q_full[b], (last / C::QB) & 1);
     }
-  for (uint32_t st = 0; st < static_cast<uint32_t>(C::NVS); ++st)
+  for (uint32_t st = 0; st < static_cast<uint32_t>(C::KS); ++st)
+    if (k_loads > st) {
+      const uint32_t last = st + C::KS * ((k_loads - 1 - st) / C::KS);
+      wait_drain(&B.k_full[st], (last / C::KS) & 1);
+    }
+  for (uint32_t st = 0; st < static_cast<uint32_t>(C::VS); ++st)
     if (v_loads > st) {
-      const uint32_t last = st + C::NVS * ((v_loads - 1 - st) / C::NVS);
-      wait_drain(&ctl->v_full[st], (last / C::NVS) & 1);
+      const uint32_t last = st + C::VS * ((v_loads - 1 - st) / C::VS);
+      wait_drain(&B.v_full[st], (last / C::VS) & 1);
     }
 }
 
 // ---------------------------------------------------------------- MMA issuer
-// Order: S(0) of each slot, then per slot in turn O += P(j) V(j) and the
-// slot's next S (step j+1 of its tile, or step 0 of its next tile).  MMAs of
-// one thread complete in issue order, so a slot's next S overwrites S/P only
-// after the P V that reads P, and the commit of a slot's S also reports that
-// its previous P V has finished (the softmax relies on this to rescale O).
+// One thread serves both slots without blocking on either: each pass it
+// tries, per slot, the next O += P V and the next S = Q K^T, and issues those
+// whose barriers have completed (non-blocking tests).  Per slot, S of step
+// g+1 runs at most one step ahead of the P V of step g.  With P written over
+// S, a slot's next S is issued only after its P V; MMAs of one thread
+// complete in issue order, so S overwrites P only after the P V has read it,
+// and the commit of S also reports that the previous P V has finished.  With
+// P in its own columns, a slot's next S waits only until the softmax has
+// loaded the current scores (s_free), and each P V commits pv_done.
+struct PStep {          // a step whose S is issued and whose P V is not
+  int buf;
+  bool first, last;
+};
+
+struct MmaSlot {        // the MMA issuer's state for one slot (kept in registers)
+  int t = 0;            // tile-info entry of the S side's tile
+  int qsteps = 0, qj = 0;  // steps of that tile, next S step (qj == qsteps: next tile)
+  bool done = false;    // the S side has seen the end of the slot's work
+  uint32_t q_uses = 0, k_cons = 0, v_cons = 0, qk_issued = 0, p_seen = 0;
+  PStep front, back;    // P V queue (at most two steps)
+  int pcount = 0;
+};
+
 template <int BS, int D>
 __device__ void mma_role(const FwdArgs& a, uint8_t* smem, Ctrl* ctl, uint32_t tmem) {
   using C = Cfg<BS, D>;
   constexpr uint32_t kIdescQK = idesc_bf16_f32(128, C::NK, false, false);  // Q, K K-major
   constexpr uint32_t kIdescPV = idesc_bf16_f32(128, D, false, true);       // V MN-major
-  const uint32_t q_base = smem_u32(smem + C::OFF_Q);
-  const uint32_t k_base = smem_u32(smem + C::OFF_K);
-  const uint32_t v_base = smem_u32(smem + C::OFF_V);
-  uint32_t k_cons = 0, v_cons = 0;
-  uint32_t q_uses[kSlots] = {0, 0}, p_seen[kSlots] = {0, 0};
-  int t[kSlots] = {0, 0}, steps[kSlots] = {0, 0}, j[kSlots] = {0, 0};
-  bool active[kSlots] = {true, true};
-  bool ok = true;
+  const uint32_t sbase = smem_u32(smem);
+  MmaSlot sl0, sl1;
 
-  auto next_tile_of = [&](int s) -> bool {
-    for (;;) {
-      const int buf = t[s] & 1;
-      if (!wait_bounded(&ctl->t_full[s][buf], (t[s] >> 1) & 1, &ctl->abort)) return false;
+  // Next S = Q K^T of slot s, if every input is ready: 1 issued (or an empty
+  // tile skipped), 0 not ready, -1 inconsistent tile info.
+  auto try_qk = [&](MmaSlot& st, int s) -> int {
+    SlotBars& B = ctl->sb[s];
+    if (st.done) return 0;
+    if (st.qj == st.qsteps) {  // the next tile
+      const int buf = st.t % kTiRing;
+      if (!mbar_test_wait(&B.t_full[buf], (st.t / kTiRing) & 1)) return 0;
       const long long tile = ctl->info[s][buf].tile;
       const int n = ctl->info[s][buf].n;
       if (tile < 0) {
-        active[s] = false;
-        return true;
+        st.done = true;
+        return 0;
       }
+      if (tile >= a.num_tiles || n > a.M) return -1;  // never for a consistent schedule
       if (n == 0) {
-        mbar_arrive(&ctl->t_empty[s][buf]);
-        ++t[s];
-        continue;
+        mbar_arrive(&B.t_empty[buf]);
+        ++st.t;
+        return 1;
       }
-      steps[s] = (n + C::BPS - 1) / C::BPS;
-      j[s] = 0;
-      return true;
+      st.qsteps = (n + C::BPS - 1) / C::BPS;
+      st.qj = 0;
     }
-  };
-  auto issue_qk = [&](int s) -> bool {
-    const uint32_t qb = q_uses[s] % C::QB;
-    if (j[s] == 0 &&
-        !wait_bounded(&ctl->q_full[s][qb], (q_uses[s] / C::QB) & 1, &ctl->abort))
-      return false;
-    const uint32_t ks = k_cons % C::NKS;
-    if (!wait_bounded(&ctl->k_full[ks], (k_cons / C::NKS) & 1, &ctl->abort)) return false;
+    if (!C::SEP_P && st.pcount > 0) return 0;  // P lives in S: its P V goes first
+    const uint32_t qb = st.q_uses % C::QB;
+    if (st.qj == 0 && !mbar_test_wait(&B.q_full[qb], (st.q_uses / C::QB) & 1)) return 0;
+    if (C::SEP_P && st.qk_issued > 0 && !mbar_test_wait(&B.s_free, (st.qk_issued - 1) & 1))
+      return 0;
+    const uint32_t ks = st.k_cons % C::KS;
+    if (!mbar_test_wait(&B.k_full[ks], (st.k_cons / C::KS) & 1)) return 0;
     tc_fence_after();
-    // Descriptors of consecutive K=16 slices differ only in the start
-    // address field (address >> 4), so they are a base plus a constant.
-    const uint64_t ad0 = sdesc_sw128(q_base + (s * C::QB + qb) * C::Q_BYTES, 16, 1024);
-    const uint64_t bd0 = sdesc_sw128(k_base + ks * C::CH_BYTES, 16, 1024);
-#pragma unroll
-    for (int kk = 0; kk < D / 16; ++kk) {
-      const uint32_t off = ((kk >> 2) * (C::TM * 128) + (kk & 3) * 32) >> 4;  // TM == NK
-      umma_bf16_ss(tmem + s * 128, ad0 + off, bd0 + off, kIdescQK, kk > 0 ? 1u : 0u);
+    const uint64_t ad = sdesc_sw128(sbase + C::off_q(s) + qb * C::Q_BYTES, 16, 1024);
+    const uint64_t bd = sdesc_sw128(sbase + C::off_k(s) + ks * C::CH_BYTES, 16, 1024);
+    umma_qk_chain<D / 16>(tmem + s * 128, static_cast<uint32_t>(ad), static_cast<uint32_t>(ad >> 32),
+                          static_cast<uint32_t>(bd), static_cast<uint32_t>(bd >> 32), kIdescQK);
+    umma_commit(&B.k_empty[ks]);
+    umma_commit(&B.s_full);
+    PStep e;
+    e.buf = st.t % kTiRing;
+    e.first = st.qj == 0;
+    e.last = st.qj == st.qsteps - 1;
+    if (e.last) {
+      umma_commit(&B.q_empty[qb]);
+      ++st.q_uses;
+      ++st.t;
     }
-    umma_commit(&ctl->k_empty[ks]);
-    umma_commit(&ctl->s_full[s]);
-    if (j[s] == steps[s] - 1) {
-      umma_commit(&ctl->q_empty[s][qb]);
-      ++q_uses[s];
-    }
-    ++k_cons;
-    return true;
+    ++st.qj;
+    ++st.k_cons;
+    ++st.qk_issued;
+    if (st.pcount == 0) st.front = e; else st.back = e;
+    ++st.pcount;
+    return 1;
   };
-  auto issue_pv = [&](int s) -> bool {
-    if (!wait_bounded(&ctl->p_full[s], p_seen[s] & 1, &ctl->abort)) return false;
-    ++p_seen[s];
-    const uint32_t vs = v_cons % C::NVS;
-    if (!wait_bounded(&ctl->v_full[vs], (v_cons / C::NVS) & 1, &ctl->abort)) return false;
+  // Next O += P V of slot s, if its P and V are ready.
+  auto try_pv = [&](MmaSlot& st, int s) -> int {
+    SlotBars& B = ctl->sb[s];
+    if (st.pcount == 0) return 0;
+    if (!mbar_test_wait(&B.p_full, st.p_seen & 1)) return 0;
+    const uint32_t vs = st.v_cons % C::VS;
+    if (!mbar_test_wait(&B.v_full[vs], (st.v_cons / C::VS) & 1)) return 0;
     tc_fence_after();
-    const uint64_t bd0 = sdesc_sw128(v_base + vs * C::CH_BYTES, C::NK * 128, 1024);
-    const uint32_t a0 = tmem + s * 128;
-    const uint32_t d0 = tmem + C::TMEM_O + s * D;
-#pragma unroll
-    for (int kk = 0; kk < C::NK / 16; ++kk)  // P of keys 16kk..16kk+15: TMEM columns 8kk..8kk+7
-      umma_bf16_ts(d0, a0 + kk * 8, bd0 + ((kk * 16 * 128) >> 4), kIdescPV,
-                   (j[s] > 0 || kk > 0) ? 1u : 0u);
-    umma_commit(&ctl->v_empty[vs]);
-    ++v_cons;
-    return true;
+    const PStep e = st.front;
+    // P of keys 16kk..16kk+15 sits in TMEM columns p_col + 8kk .. +7.
+    const uint64_t bd = sdesc_sw128(sbase + C::off_v(s) + vs * C::CH_BYTES, C::NK * 128, 1024);
+    umma_pv_chain8(tmem + C::TMEM_O + s * D, tmem + C::p_col(s), static_cast<uint32_t>(bd),
+                   static_cast<uint32_t>(bd >> 32), kIdescPV, e.first ? 0u : 1u);
+    umma_commit(&B.v_empty[vs]);
+    if (C::SEP_P) umma_commit(&B.pv_done);
+    if (e.last) {
+      umma_commit(&B.o_full);
+      mbar_arrive(&B.t_empty[e.buf]);
+    }
+    ++st.p_seen;
+    ++st.v_cons;
+    st.front = st.back;
+    --st.pcount;
+    return 1;
   };
 
-  for (int s = 0; ok && s < kSlots; ++s) {
-    ok = next_tile_of(s);
-    if (ok && active[s]) ok = issue_qk(s);
-  }
-  while (ok && (active[0] || active[1])) {
-    for (int s = 0; ok && s < kSlots; ++s) {
-      if (!active[s]) continue;
-      ok = issue_pv(s);
-      if (!ok) break;
-      if (j[s] == steps[s] - 1) {
-        umma_commit(&ctl->o_full[s]);
-        mbar_arrive(&ctl->t_empty[s][t[s] & 1]);
-        ++t[s];
-        ok = next_tile_of(s);
-        if (ok && active[s]) ok = issue_qk(s);
-      } else {
-        ++j[s];
-        ok = issue_qk(s);
+  long long idle_since = clock64();
+  while (!(sl0.done && sl0.pcount == 0 && sl1.done && sl1.pcount == 0)) {
+    const int r0 = try_pv(sl0, 0), r1 = try_qk(sl0, 0);
+    const int r2 = try_pv(sl1, 1), r3 = try_qk(sl1, 1);
+    if (r1 < 0 || r3 < 0) {
+      atomicOr(&g_status, BSA_STATUS_INTERNAL);
+      ctl->abort.v = 1;
+      break;
+    }
+    if (r0 | r1 | r2 | r3) {
+      idle_since = clock64();
+    } else {
+      if (ctl->abort.v) break;
+      __nanosleep(32);  // leave the issue slots of this sub-partition to the softmax warps
+      if (clock64() - idle_since > kWaitLimitCycles) {
+        atomicOr(&g_status, BSA_STATUS_TIMEOUT);
+        ctl->abort.v = 1;
+        break;
       }
     }
   }
@@ -588,17 +576,19 @@ __device__ void mma_role(const FwdArgs& a, uint8_t* smem, Ctrl* ctl, uint32_t tm
 }
 
 // ------------------------------------------------------- softmax warpgroups
-// Warpgroup s: thread i owns query row i of slot s's tile.  Per step it loads
-// the scores of the blocks its row holds, takes the running maximum (the
-// rescale of O is lazy: only when the maximum grows by more than 2^8), writes
-// P over the first 64 score columns, and at the end of the tile stores
-// O / l and the LSE.  Every TMEM access here waits for itself inside one asm
+// Warpgroup s: thread i owns query row i of slot s's tile.  A step is taken
+// in two halves of 64 score columns: load the blocks the row holds, scale,
+// mask the diagonal block of a causal tile, and keep a running maximum; the
+// rescale is lazy (only when the maximum grows by more than 2^8), and when
+// the second half raises it, the first half's P is rescaled in place.  P (bf16
+// pairs) goes to the slot's P columns; at the end of the tile O / l and the
+// LSE are stored.  Every TMEM access here waits for itself inside one asm
 // statement (see sm100_ptx.cuh).
 template <int BS, int D>
 __device__ void softmax_role(int s, const FwdArgs& a, Ctrl* ctl, const uint32_t* bitmaps,
                              uint32_t tmem) {
   using C = Cfg<BS, D>;
-  constexpr int GPB = BS / 32 < 1 ? 1 : BS / 32;  // 32-column groups per block
+  constexpr int GPB = BS / 32;                   // 32-column groups per block
   const int wq = (threadIdx.x >> 5) & 3;         // TMEM lane quadrant
   const int lane = threadIdx.x & 31;
   const int row = wq * 32 + lane;                // query row of the tile
@@ -606,19 +596,28 @@ __device__ void softmax_role(int s, const FwdArgs& a, Ctrl* ctl, const uint32_t*
   const int qq = row % BS;                       // position inside that block row
   const uint32_t t_lane = tmem + (static_cast<uint32_t>(wq * 32) << 16);
   const uint32_t t_s = t_lane + s * 128;
+  const uint32_t t_p = t_lane + C::p_col(s);
   const uint32_t t_o = t_lane + C::TMEM_O + s * D;
   const float sl2 = a.scale_log2;
   constexpr float kNegInf = -INFINITY;
   const int W = a.W;
+  SlotBars& B = ctl->sb[s];
   uint32_t s_seen = 0, o_seen = 0;
 
   for (int t = 0;; ++t) {
-    const int buf = t & 1;
-    if (!warp_wait(&ctl->t_full[s][buf], (t >> 1) & 1, &ctl->abort)) return;
+    const int buf = t % kTiRing;
+    if (!warp_wait(&B.t_full[buf], (t / kTiRing) & 1, &ctl->abort)) return;
     const long long tile = ctl->info[s][buf].tile;
     const int n = ctl->info[s][buf].n;
     if (tile < 0) return;
-    const uint32_t* bm = bitmaps + (s * 2 + buf) * bitmap_words<BS>(W);
+    if (tile >= a.num_tiles || n > a.M) {     // never for a consistent schedule
+      if (lane == 0) {
+        atomicOr(&g_status, BSA_STATUS_INTERNAL);
+        ctl->abort.v = 1;
+      }
+      return;
+    }
+    const uint32_t* bm = bitmaps + (s * kTiRing + buf) * bitmap_words<BS>(W);
     const int r_sub = static_cast<int>(tile % a.G) * C::R + sub;
     const bool row_ok = r_sub < a.M;
 
@@ -637,87 +636,124 @@ __device__ void softmax_role(int s, const FwdArgs& a, Ctrl* ctl, const uint32_t*
         if (row_ok && jb >= 0 && ((bm[sub * W + (jb >> 5)] >> (jb & 31)) & 1u)) own |= gm;
         if (a.causal && jb == r_sub) diag |= gm;
       }
-      if (!warp_wait(&ctl->s_full[s], s_seen & 1, &ctl->abort)) return;
-      ++s_seen;
+      diag &= own;
+      if (!warp_wait(&B.s_full, s_seen & 1, &ctl->abort)) return;
+      const uint32_t g_step = s_seen++;        // steps of this slot before this one
       tc_fence_after();
-      uint32_t u[128];
-      tmem_ld128_groups_wait(t_s, own, u);
-
-      // Scaled scores (log2 units), the causal mask, and the row maximum.
-      float mx = kNegInf;
+      float osc = 1.f;                         // factor O must take before this step's P V
+#pragma unroll 1
+      for (int h = 0; h < 2; ++h) {
+        const uint32_t ho = (own >> (2 * h)) & 3u, hd = (diag >> (2 * h)) & 3u;
+        float x[64];
+        __syncwarp();
+        if (ho == 3u) {
+          tmem_ld64_wait(t_s + 64 * h, x);
+        } else if (ho == 1u) {
+          tmem_ld32lo_wait(t_s + 64 * h, x);
+        } else if (ho == 2u) {
+          tmem_ld32hi_wait(t_s + 64 * h + 32, x);
+        }
+        if (C::SEP_P && h == 1) {              // the scores are in registers: S may be rewritten
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&B.s_free);
+        }
+        float hm = kNegInf;
 #pragma unroll
-      for (int gi = 0; gi < 4; ++gi) {
-        if (!((own >> gi) & 1u)) continue;
-        const bool dg = (diag >> gi) & 1u;
-        float m0 = kNegInf, m1 = kNegInf;
+        for (int gi = 0; gi < 2; ++gi) {
+          if (!((ho >> gi) & 1u)) continue;
 #pragma unroll
-        for (int c = 0; c < 32; c += 2) {
-          float x0 = __uint_as_float(u[gi * 32 + c]) * sl2;
-          float x1 = __uint_as_float(u[gi * 32 + c + 1]) * sl2;
-          if (dg) {  // key after the query (diagonal block only)
-            const int kc = (gi * 32 + c) % BS;
-            if (kc > qq) x0 = kNegInf;
-            if (kc + 1 > qq) x1 = kNegInf;
+          for (int c = 0; c < 32; c += 2) mul2(x[gi * 32 + c], x[gi * 32 + c + 1], sl2);
+          if ((hd >> gi) & 1u) {               // keys after the query (diagonal block only)
+#pragma unroll
+            for (int c = 0; c < 32; ++c)
+              if ((64 * h + gi * 32 + c) % BS > qq) x[gi * 32 + c] = kNegInf;
           }
-          u[gi * 32 + c] = __float_as_uint(x0);
-          u[gi * 32 + c + 1] = __float_as_uint(x1);
-          m0 = fmaxf(m0, x0);
-          m1 = fmaxf(m1, x1);
-        }
-        mx = fmaxf(mx, fmaxf(m0, m1));
-      }
-
-      // Lazy rescale: the running maximum moves only when the step's maximum
-      // exceeds it by more than the threshold (P stays <= 2^8 otherwise).
-      float factor = 1.f;
-      bool need_rescale = false;
-      if (mx > m_used + kRescaleThreshold) {
-        if (m_used != kNegInf) {
-          need_rescale = true;
-          factor = ex2_approx(m_used - mx);
-        }
-        m_used = mx;
-      }
-      l *= factor;
-
-      // P = 2^(x - m_used) in bf16 pairs over the first 64 score columns.
-      const float mu = m_used == kNegInf ? 0.f : m_used;
-      float r0 = 0.f, r1 = 0.f;
-      uint32_t pk[64];
+          float ma = kNegInf, mb = kNegInf;
 #pragma unroll
-      for (int gi = 0; gi < 4; ++gi) {
-        if ((own >> gi) & 1u) {
-#pragma unroll
-          for (int c = 0; c < 32; c += 2) {
-            const float p0 = ex2_approx(__uint_as_float(u[gi * 32 + c]) - mu);
-            const float p1 = ex2_approx(__uint_as_float(u[gi * 32 + c + 1]) - mu);
-            r0 += p0;
-            r1 += p1;
-            pk[gi * 16 + c / 2] = pack_bf16x2(p0, p1);
+          for (int c = 0; c < 32; c += 4) {
+            ma = max3f(ma, x[gi * 32 + c], x[gi * 32 + c + 1]);
+            mb = max3f(mb, x[gi * 32 + c + 2], x[gi * 32 + c + 3]);
           }
-        } else {
-#pragma unroll
-          for (int i = 0; i < 16; ++i) pk[gi * 16 + i] = 0u;
+          hm = max3f(hm, ma, mb);
         }
-      }
-      l += r0 + r1;
-      tmem_st64_wait(t_s, pk);
-      // O holds the P V of every earlier step (this step's S being ready
-      // means the previous P V has completed); bring it to the new maximum
-      // before this step's P V adds to it.
-      if (__any_sync(0xffffffffu, need_rescale)) {
+        // Lazy rescale: the running maximum moves only when it is exceeded by
+        // more than the threshold (P stays <= 2^8 otherwise).
+        const bool need = hm > m_used + kRescaleThreshold;
+        if (__any_sync(0xffffffffu, need)) {
+          float f = 1.f;
+          if (need) {
+            if (m_used != kNegInf) f = ex2_approx(m_used - hm);
+            m_used = hm;
+          }
+          l *= f;
+          osc *= f;
+          if (h == 1 && __any_sync(0xffffffffu, f != 1.f)) {
+            // The first half's P was taken against the old maximum.
+            uint32_t w[32];
+            __syncwarp();
+            tmem_ld32_wait(t_p, w);
 #pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const float lo = __uint_as_float(w[i] << 16) * f;
+              const float hi = __uint_as_float(w[i] & 0xffff0000u) * f;
+              w[i] = pack_bf16x2(lo, hi);
+            }
+            tmem_st32_wait(t_p, w);
+          }
+        }
+        // P = 2^(x - m_used) in bf16 pairs: keys 64h .. 64h+63 to P columns 32h .. 32h+31.
+        const float nmu = m_used == kNegInf ? 0.f : -m_used;
+        float sa = 0.f, sb = 0.f, sc = 0.f, sd = 0.f;
+        uint32_t pk[32];
+#pragma unroll
+        for (int gi = 0; gi < 2; ++gi) {
+          if ((ho >> gi) & 1u) {
+#pragma unroll
+            for (int c = 0; c < 32; c += 4) {
+              float d0 = x[gi * 32 + c], d1 = x[gi * 32 + c + 1];
+              float d2 = x[gi * 32 + c + 2], d3 = x[gi * 32 + c + 3];
+              add2(d0, d1, nmu);
+              add2(d2, d3, nmu);
+              const float p0 = ex2_approx(d0), p1 = ex2_approx(d1);
+              const float p2 = ex2_approx(d2), p3 = ex2_approx(d3);
+              acc2(sa, sb, p0, p1);
+              acc2(sc, sd, p2, p3);
+              pk[gi * 16 + c / 2] = pack_bf16x2(p0, p1);
+              pk[gi * 16 + c / 2 + 1] = pack_bf16x2(p2, p3);
+            }
+          } else {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) pk[gi * 16 + i] = 0u;
+          }
+        }
+        l += (sa + sb) + (sc + sd);
+        if (C::SEP_P && h == 0 && g_step > 0) {
+          // P is about to be rewritten and O may be rescaled: the previous
+          // P V of this slot must have finished.
+          if (!warp_wait(&B.pv_done, (g_step - 1) & 1, &ctl->abort)) return;
+          tc_fence_after();
+        }
+        __syncwarp();
+        tmem_st32_wait(t_p + 32 * h, pk);
+      }
+      // O holds the P V of every earlier step (with P over S, this step's S
+      // being ready means the previous P V has completed); bring it to the
+      // new maximum before this step's P V adds to it.
+      if (__any_sync(0xffffffffu, osc != 1.f)) {
+#pragma unroll 1
         for (int c0 = 0; c0 < D; c0 += 32) {
           uint32_t w[32];
+          __syncwarp();
           tmem_ld32_wait(t_o + c0, w);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) w[i] = __float_as_uint(__uint_as_float(w[i]) * factor);
+          for (int i = 0; i < 32; ++i) w[i] = __float_as_uint(__uint_as_float(w[i]) * osc);
           tmem_st32_wait(t_o + c0, w);
         }
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&ctl->p_full[s]);
+      if (lane == 0) mbar_arrive(&B.p_full);
     }
 
     // Epilogue: O / l in bf16 and LSE = (m + log2 l) ln 2, once the last P V
@@ -726,15 +762,16 @@ __device__ void softmax_role(int s, const FwdArgs& a, Ctrl* ctl, const uint32_t*
     const long long qtok = (tile - bh * a.G) * C::TM + row;
     uint4* orow = reinterpret_cast<uint4*>(a.O + (bh * a.N + qtok) * D);
     if (n > 0) {
-      if (!warp_wait(&ctl->o_full[s], o_seen & 1, &ctl->abort)) return;
+      if (!warp_wait(&B.o_full, o_seen & 1, &ctl->abort)) return;
       ++o_seen;
       tc_fence_after();
     }
     const float inv = l > 0.f ? 1.f / l : 0.f;
-#pragma unroll
+#pragma unroll 1
     for (int c0 = 0; c0 < D; c0 += 32) {
       uint32_t w[32];
       if (n > 0) {
+        __syncwarp();
         tmem_ld32_wait(t_o + c0, w);
       } else {
 #pragma unroll
@@ -756,7 +793,7 @@ __device__ void softmax_role(int s, const FwdArgs& a, Ctrl* ctl, const uint32_t*
       a.LSE[bh * a.N + qtok] = l > 0.f ? (m_used + __log2f(l)) * 0.69314718055994531f : kNegInf;
     tc_fence_before();
     __syncwarp();
-    if (lane == 0) mbar_arrive(&ctl->t_empty[s][buf]);
+    if (lane == 0) mbar_arrive(&B.t_empty[buf]);
   }
 }
 
@@ -774,21 +811,24 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kSlots; ++s) {
-      for (int b = 0; b < 2; ++b) {
-        mbar_init(&ctl->t_full[s][b], 1);
-        mbar_init(&ctl->t_empty[s][b], 4 + 2);  // the slot's softmax warps, the loader, the MMA issuer
-        mbar_init(&ctl->q_full[s][b], 1);
-        mbar_init(&ctl->q_empty[s][b], 1);
+      SlotBars& B = ctl->sb[s];
+      for (int b = 0; b < kTiRing; ++b) {
+        mbar_init(&B.t_full[b], 1);
+        mbar_init(&B.t_empty[b], 4 + 2);  // the slot's softmax warps, its producer, the MMA issuer
       }
-      mbar_init(&ctl->s_full[s], 1);
-      mbar_init(&ctl->p_full[s], 4);
-      mbar_init(&ctl->o_full[s], 1);
-    }
-    for (int i = 0; i < 4; ++i) {
-      mbar_init(&ctl->k_full[i], 1);
-      mbar_init(&ctl->k_empty[i], 1);
-      mbar_init(&ctl->v_full[i], 1);
-      mbar_init(&ctl->v_empty[i], 1);
+      for (int b = 0; b < 2; ++b) {
+        mbar_init(&B.q_full[b], 1);
+        mbar_init(&B.q_empty[b], 1);
+        mbar_init(&B.k_full[b], 1);
+        mbar_init(&B.k_empty[b], 1);
+        mbar_init(&B.v_full[b], 1);
+        mbar_init(&B.v_empty[b], 1);
+      }
+      mbar_init(&B.s_full, 1);
+      mbar_init(&B.p_full, 4);
+      mbar_init(&B.o_full, 1);
+      mbar_init(&B.s_free, 4);
+      mbar_init(&B.pv_done, 1);
     }
     mbar_init(&ctl->final_bar, 1);
     ctl->abort.v = 0;
@@ -804,26 +844,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = ctl->tmem_base;
 
-  // Registers: the launch gives every thread kLaunchRegs; the softmax
-  // warpgroups (a full score row per thread) take kSoftRegs, warpgroup 2
-  // (the four single-warp roles) gives its share back.  Each warpgroup
-  // executes its reallocation at one point, all four warps together.
-  if (warp < 4 * kSlots) {
-    reg_alloc_inc<kSoftRegs>();
-  } else {
-    reg_alloc_dec<kOtherRegs>();
-  }
   if (warp < 4 * kSlots) {
     softmax_role<BS, D>(warp >> 2, args, ctl, bitmaps, tmem);
     __syncwarp();
-  } else if (warp == kLoadWarp) {
-    load_role<BS, D>(&tmQ, &tmK, &tmV, args, smem, ctl, bitmaps);
+  } else if (warp == kProdWarp || warp == kProdWarp + 2) {
+    produce_role<BS, D>((warp - kProdWarp) >> 1, &tmQ, &tmK, &tmV, args, smem, ctl, bitmaps);
     __syncwarp();
   } else if (warp == kMmaWarp) {
     if ((threadIdx.x & 31) == 0) mma_role<BS, D>(args, smem, ctl, tmem);
     __syncwarp();
-  } else {
-    build_role<BS, D>(warp - kBuildWarp, args, ctl, bitmaps);
   }
 
   tc_fence_before();

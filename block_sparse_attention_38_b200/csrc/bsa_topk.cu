@@ -215,7 +215,8 @@ extern "C" int bsa_topk_pattern(const void* Q, const void* K, int BH, int N, int
 // bsa_topk_pattern_static: the same selection with its fp64 workspace in a
 // fixed scratch area of this library instead of caller memory.  Every device
 // gets its own copy of the array when the library's module loads there; its
-// address is looked up once per device, on the first call.  No element of the
+// address is looked up once per device, on the first call, and kept for the
+// life of the process (a device reset leaves it stale).  No element of the
 // scratch needs to start at zero: the means kernel writes every element the
 // selection then reads, within the same call.  Two calls that overlap in time
 // on one device share the area and race.

@@ -34,6 +34,19 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
                : "memory");
 }
 
+// Non-blocking: true when the phase of parity `parity` has completed.
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t done;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(done)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return done != 0;
+}
+
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t done;
   asm volatile(
@@ -55,6 +68,14 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, u
       " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(dst)),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2)
       : "memory");
+}
+
+// 3-D tiled prefetch of a box into L2 (no shared memory, no completion).
+__device__ __forceinline__ void tma_prefetch_3d(const CUtensorMap* map, int c0, int c1, int c2) {
+  asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(c0), "r"(c1), "r"(c2)
+               : "memory");
 }
 
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
@@ -121,24 +142,34 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
 // one statement the compiler cannot place a spill or another value in them
 // in between.
 
-// Loads the 32-column groups g (bit g of `groups`, uniform over the warp) of
-// the 128 columns at `taddr` into r[32g .. 32g+31] and waits for them; the
-// registers of groups not loaded are left undefined.
-__device__ __forceinline__ void tmem_ld128_groups_wait(uint32_t taddr, uint32_t groups,
-                                                       uint32_t (&r)[128]) {
+
+// Loads the 64 columns at `taddr` into r as fp32 and waits for them.  The
+// outputs are early-clobber, so none shares a register with the address.
+__device__ __forceinline__ void tmem_ld64_wait(uint32_t taddr, float (&r)[64]) {
   asm volatile(
-      "{\n\t.reg .pred p<4>;\n\t.reg .b32 t;\n\t"
-      "and.b32 t, %129, 1;\n\tsetp.ne.b32 p0, t, 0;\n\t"
-      "and.b32 t, %129, 2;\n\tsetp.ne.b32 p1, t, 0;\n\t"
-      "and.b32 t, %129, 4;\n\tsetp.ne.b32 p2, t, 0;\n\t"
-      "and.b32 t, %129, 8;\n\tsetp.ne.b32 p3, t, 0;\n\t"
-      "@p0 tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%128+0];\n\t"
-      "@p1 tcgen05.ld.sync.aligned.32x32b.x32.b32 {%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%128+32];\n\t"
-      "@p2 tcgen05.ld.sync.aligned.32x32b.x32.b32 {%64,%65,%66,%67,%68,%69,%70,%71,%72,%73,%74,%75,%76,%77,%78,%79,%80,%81,%82,%83,%84,%85,%86,%87,%88,%89,%90,%91,%92,%93,%94,%95}, [%128+64];\n\t"
-      "@p3 tcgen05.ld.sync.aligned.32x32b.x32.b32 {%96,%97,%98,%99,%100,%101,%102,%103,%104,%105,%106,%107,%108,%109,%110,%111,%112,%113,%114,%115,%116,%117,%118,%119,%120,%121,%122,%123,%124,%125,%126,%127}, [%128+96];\n\t"
+      "{\n\ttcgen05.ld.sync.aligned.32x32b.x64.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%64];\n\t"
       "tcgen05.wait::ld.sync.aligned;\n\t}"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]), "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]), "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]), "=r"(r[48]), "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]), "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63]), "=r"(r[64]), "=r"(r[65]), "=r"(r[66]), "=r"(r[67]), "=r"(r[68]), "=r"(r[69]), "=r"(r[70]), "=r"(r[71]), "=r"(r[72]), "=r"(r[73]), "=r"(r[74]), "=r"(r[75]), "=r"(r[76]), "=r"(r[77]), "=r"(r[78]), "=r"(r[79]), "=r"(r[80]), "=r"(r[81]), "=r"(r[82]), "=r"(r[83]), "=r"(r[84]), "=r"(r[85]), "=r"(r[86]), "=r"(r[87]), "=r"(r[88]), "=r"(r[89]), "=r"(r[90]), "=r"(r[91]), "=r"(r[92]), "=r"(r[93]), "=r"(r[94]), "=r"(r[95]), "=r"(r[96]), "=r"(r[97]), "=r"(r[98]), "=r"(r[99]), "=r"(r[100]), "=r"(r[101]), "=r"(r[102]), "=r"(r[103]), "=r"(r[104]), "=r"(r[105]), "=r"(r[106]), "=r"(r[107]), "=r"(r[108]), "=r"(r[109]), "=r"(r[110]), "=r"(r[111]), "=r"(r[112]), "=r"(r[113]), "=r"(r[114]), "=r"(r[115]), "=r"(r[116]), "=r"(r[117]), "=r"(r[118]), "=r"(r[119]), "=r"(r[120]), "=r"(r[121]), "=r"(r[122]), "=r"(r[123]), "=r"(r[124]), "=r"(r[125]), "=r"(r[126]), "=r"(r[127])
-      : "r"(taddr), "r"(groups)
+      : "=&f"(r[0]), "=&f"(r[1]), "=&f"(r[2]), "=&f"(r[3]), "=&f"(r[4]), "=&f"(r[5]), "=&f"(r[6]), "=&f"(r[7]), "=&f"(r[8]), "=&f"(r[9]), "=&f"(r[10]), "=&f"(r[11]), "=&f"(r[12]), "=&f"(r[13]), "=&f"(r[14]), "=&f"(r[15]), "=&f"(r[16]), "=&f"(r[17]), "=&f"(r[18]), "=&f"(r[19]), "=&f"(r[20]), "=&f"(r[21]), "=&f"(r[22]), "=&f"(r[23]), "=&f"(r[24]), "=&f"(r[25]), "=&f"(r[26]), "=&f"(r[27]), "=&f"(r[28]), "=&f"(r[29]), "=&f"(r[30]), "=&f"(r[31]), "=&f"(r[32]), "=&f"(r[33]), "=&f"(r[34]), "=&f"(r[35]), "=&f"(r[36]), "=&f"(r[37]), "=&f"(r[38]), "=&f"(r[39]), "=&f"(r[40]), "=&f"(r[41]), "=&f"(r[42]), "=&f"(r[43]), "=&f"(r[44]), "=&f"(r[45]), "=&f"(r[46]), "=&f"(r[47]), "=&f"(r[48]), "=&f"(r[49]), "=&f"(r[50]), "=&f"(r[51]), "=&f"(r[52]), "=&f"(r[53]), "=&f"(r[54]), "=&f"(r[55]), "=&f"(r[56]), "=&f"(r[57]), "=&f"(r[58]), "=&f"(r[59]), "=&f"(r[60]), "=&f"(r[61]), "=&f"(r[62]), "=&f"(r[63])
+      : "r"(taddr)
+      : "memory");
+}
+
+// Loads the 32 columns at `taddr` into r[0..31] (lo) or r[32..63] (hi) as
+// fp32 and waits for them; the other half of r is left undefined.
+__device__ __forceinline__ void tmem_ld32lo_wait(uint32_t taddr, float (&r)[64]) {
+  asm volatile(
+      "{\n\ttcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n\t"
+      "tcgen05.wait::ld.sync.aligned;\n\t}"
+      : "=&f"(r[0]), "=&f"(r[1]), "=&f"(r[2]), "=&f"(r[3]), "=&f"(r[4]), "=&f"(r[5]), "=&f"(r[6]), "=&f"(r[7]), "=&f"(r[8]), "=&f"(r[9]), "=&f"(r[10]), "=&f"(r[11]), "=&f"(r[12]), "=&f"(r[13]), "=&f"(r[14]), "=&f"(r[15]), "=&f"(r[16]), "=&f"(r[17]), "=&f"(r[18]), "=&f"(r[19]), "=&f"(r[20]), "=&f"(r[21]), "=&f"(r[22]), "=&f"(r[23]), "=&f"(r[24]), "=&f"(r[25]), "=&f"(r[26]), "=&f"(r[27]), "=&f"(r[28]), "=&f"(r[29]), "=&f"(r[30]), "=&f"(r[31])
+      : "r"(taddr)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_ld32hi_wait(uint32_t taddr, float (&r)[64]) {
+  asm volatile(
+      "{\n\ttcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n\t"
+      "tcgen05.wait::ld.sync.aligned;\n\t}"
+      : "=&f"(r[32]), "=&f"(r[33]), "=&f"(r[34]), "=&f"(r[35]), "=&f"(r[36]), "=&f"(r[37]), "=&f"(r[38]), "=&f"(r[39]), "=&f"(r[40]), "=&f"(r[41]), "=&f"(r[42]), "=&f"(r[43]), "=&f"(r[44]), "=&f"(r[45]), "=&f"(r[46]), "=&f"(r[47]), "=&f"(r[48]), "=&f"(r[49]), "=&f"(r[50]), "=&f"(r[51]), "=&f"(r[52]), "=&f"(r[53]), "=&f"(r[54]), "=&f"(r[55]), "=&f"(r[56]), "=&f"(r[57]), "=&f"(r[58]), "=&f"(r[59]), "=&f"(r[60]), "=&f"(r[61]), "=&f"(r[62]), "=&f"(r[63])
+      : "r"(taddr)
       : "memory");
 }
 
@@ -156,7 +187,7 @@ __device__ __forceinline__ void tmem_ld32_wait(uint32_t taddr, uint32_t (&r)[32]
   asm volatile(
       "{\n\ttcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n\t"
       "tcgen05.wait::ld.sync.aligned;\n\t}"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "=&r"(r[0]), "=&r"(r[1]), "=&r"(r[2]), "=&r"(r[3]), "=&r"(r[4]), "=&r"(r[5]), "=&r"(r[6]), "=&r"(r[7]), "=&r"(r[8]), "=&r"(r[9]), "=&r"(r[10]), "=&r"(r[11]), "=&r"(r[12]), "=&r"(r[13]), "=&r"(r[14]), "=&r"(r[15]), "=&r"(r[16]), "=&r"(r[17]), "=&r"(r[18]), "=&r"(r[19]), "=&r"(r[20]), "=&r"(r[21]), "=&r"(r[22]), "=&r"(r[23]), "=&r"(r[24]), "=&r"(r[25]), "=&r"(r[26]), "=&r"(r[27]), "=&r"(r[28]), "=&r"(r[29]), "=&r"(r[30]), "=&r"(r[31])
       : "r"(taddr)
       : "memory");
 }
@@ -193,6 +224,92 @@ __device__ __forceinline__ void umma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, u
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
       "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// One step's chain of K=16 MMAs in a single asm statement, so the issuing
+// thread runs nothing but 32-bit descriptor adds between them (the tensor
+// core idles while the issuer computes).  The start-address field of a
+// shared-memory descriptor is its low 14 bits (address >> 4); shared
+// addresses stay below 2^18 bytes, so the adds never carry out of the low word.
+
+// S (fp32, TMEM) = A B^T over K = 16*NK: A and B K-major SW128 tiles of 128
+// rows, 64-column atoms 128*128 bytes apart (descriptor lo/hi words given for
+// the first slice).  The first MMA overwrites S.
+template <int NK>
+__device__ __forceinline__ void umma_qk_chain(uint32_t d_tmem, uint32_t a_lo, uint32_t a_hi,
+                                              uint32_t b_lo, uint32_t b_hi, uint32_t idesc);
+template <>
+__device__ __forceinline__ void umma_qk_chain<4>(uint32_t d_tmem, uint32_t a_lo, uint32_t a_hi,
+                                                 uint32_t b_lo, uint32_t b_hi, uint32_t idesc) {
+  asm volatile(
+      "{\n\t.reg .pred pf, pt;\n\t.reg .b32 al, bl, one;\n\t.reg .b64 ad, bd;\n\t"
+      "mov.b32 one, 1;\n\tsetp.eq.b32 pt, one, 1;\n\tsetp.eq.b32 pf, one, 0;\n\t"
+      "add.s32 al, %1, 0;\n\tadd.s32 bl, %3, 0;\n\tmov.b64 ad, {al, %2};\n\tmov.b64 bd, {bl, %4};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %5, pf;\n\t"
+      "add.s32 al, %1, 2;\n\tadd.s32 bl, %3, 2;\n\tmov.b64 ad, {al, %2};\n\tmov.b64 bd, {bl, %4};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %5, pt;\n\t"
+      "add.s32 al, %1, 4;\n\tadd.s32 bl, %3, 4;\n\tmov.b64 ad, {al, %2};\n\tmov.b64 bd, {bl, %4};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %5, pt;\n\t"
+      "add.s32 al, %1, 6;\n\tadd.s32 bl, %3, 6;\n\tmov.b64 ad, {al, %2};\n\tmov.b64 bd, {bl, %4};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %5, pt;\n\t"
+      "}"
+      :: "r"(d_tmem), "r"(a_lo), "r"(a_hi), "r"(b_lo), "r"(b_hi), "r"(idesc)
+      : "memory");
+}
+template <>
+__device__ __forceinline__ void umma_qk_chain<8>(uint32_t d_tmem, uint32_t a_lo, uint32_t a_hi,
+                                                 uint32_t b_lo, uint32_t b_hi, uint32_t idesc) {
+  asm volatile(
+      "{\n\t.reg .pred pf, pt;\n\t.reg .b32 al, bl, one;\n\t.reg .b64 ad, bd;\n\t"
+      "mov.b32 one, 1;\n\tsetp.eq.b32 pt, one, 1;\n\tsetp.eq.b32 pf, one, 0;\n\t"
+      "add.s32 al, %1, 0;\n\tadd.s32 bl, %3, 0;\n\tmov.b64 ad, {al, %2};\n\tmov.b64 bd, {bl, %4};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %5, pf;\n\t"
+      "add.s32 al, %1, 2;\n\tadd.s32 bl, %3, 2;\n\tmov.b64 ad, {al, %2};\n\tmov.b64 bd, {bl, %4};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %5, pt;\n\t"
+      "add.s32 al, %1, 4;\n\tadd.s32 bl, %3, 4;\n\tmov.b64 ad, {al, %2};\n\tmov.b64 bd, {bl, %4};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %5, pt;\n\t"
+      "add.s32 al, %1, 6;\n\tadd.s32 bl, %3, 6;\n\tmov.b64 ad, {al, %2};\n\tmov.b64 bd, {bl, %4};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %5, pt;\n\t"
+      "add.s32 al, %1, 1024;\n\tadd.s32 bl, %3, 1024;\n\tmov.b64 ad, {al, %2};\n\tmov.b64 bd, {bl, %4};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %5, pt;\n\t"
+      "add.s32 al, %1, 1026;\n\tadd.s32 bl, %3, 1026;\n\tmov.b64 ad, {al, %2};\n\tmov.b64 bd, {bl, %4};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %5, pt;\n\t"
+      "add.s32 al, %1, 1028;\n\tadd.s32 bl, %3, 1028;\n\tmov.b64 ad, {al, %2};\n\tmov.b64 bd, {bl, %4};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %5, pt;\n\t"
+      "add.s32 al, %1, 1030;\n\tadd.s32 bl, %3, 1030;\n\tmov.b64 ad, {al, %2};\n\tmov.b64 bd, {bl, %4};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %5, pt;\n\t"
+      "}"
+      :: "r"(d_tmem), "r"(a_lo), "r"(a_hi), "r"(b_lo), "r"(b_hi), "r"(idesc)
+      : "memory");
+}
+
+// O (fp32, TMEM) (+)= P V over 128 keys: P (bf16 pairs) in TMEM, 8 columns per
+// K=16 slice from a_tmem; V an MN-major SW128 tile, 16 key rows = 2048 bytes
+// per slice.  The first MMA accumulates only if `accumulate` is non-zero.
+__device__ __forceinline__ void umma_pv_chain8(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_lo,
+                                               uint32_t b_hi, uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p0, pt;\n\t.reg .b32 bl, at, one;\n\t.reg .b64 bd;\n\t"
+      "mov.b32 one, 1;\n\tsetp.eq.b32 pt, one, 1;\n\tsetp.ne.b32 p0, %5, 0;\n\t"
+      "add.s32 at, %1, 0;\n\tadd.s32 bl, %2, 0;\n\tmov.b64 bd, {bl, %3};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [at], bd, %4, p0;\n\t"
+      "add.s32 at, %1, 8;\n\tadd.s32 bl, %2, 128;\n\tmov.b64 bd, {bl, %3};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [at], bd, %4, pt;\n\t"
+      "add.s32 at, %1, 16;\n\tadd.s32 bl, %2, 256;\n\tmov.b64 bd, {bl, %3};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [at], bd, %4, pt;\n\t"
+      "add.s32 at, %1, 24;\n\tadd.s32 bl, %2, 384;\n\tmov.b64 bd, {bl, %3};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [at], bd, %4, pt;\n\t"
+      "add.s32 at, %1, 32;\n\tadd.s32 bl, %2, 512;\n\tmov.b64 bd, {bl, %3};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [at], bd, %4, pt;\n\t"
+      "add.s32 at, %1, 40;\n\tadd.s32 bl, %2, 640;\n\tmov.b64 bd, {bl, %3};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [at], bd, %4, pt;\n\t"
+      "add.s32 at, %1, 48;\n\tadd.s32 bl, %2, 768;\n\tmov.b64 bd, {bl, %3};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [at], bd, %4, pt;\n\t"
+      "add.s32 at, %1, 56;\n\tadd.s32 bl, %2, 896;\n\tmov.b64 bd, {bl, %3};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [at], bd, %4, pt;\n\t"
+      "}"
+      :: "r"(d_tmem), "r"(a_tmem), "r"(b_lo), "r"(b_hi), "r"(idesc), "r"(accumulate)
       : "memory");
 }
 
@@ -250,18 +367,33 @@ __device__ __forceinline__ void reg_fence32(uint32_t (&r)[32]) {
   asm volatile("" : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31]));
 }
 
-// Warpgroup-wide register reallocation: every thread of the warpgroup
-// executes the same instruction; the new per-thread count is a multiple of 8.
-template <int N>
-__device__ __forceinline__ void reg_alloc_inc() {
-  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+// ------------------------------------------------------------------- math
+// Packed pairs of fp32 (one instruction for two lanes of arithmetic).
+__device__ __forceinline__ void mul2(float& a, float& b, float s) {
+  asm("{\n\t.reg .b64 x, y;\n\tmov.b64 x, {%0, %1};\n\tmov.b64 y, {%2, %2};\n\t"
+      "mul.rn.ftz.f32x2 x, x, y;\n\tmov.b64 {%0, %1}, x;\n\t}"
+      : "+f"(a), "+f"(b)
+      : "f"(s));
 }
-template <int N>
-__device__ __forceinline__ void reg_alloc_dec() {
-  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+__device__ __forceinline__ void add2(float& a, float& b, float s) {
+  asm("{\n\t.reg .b64 x, y;\n\tmov.b64 x, {%0, %1};\n\tmov.b64 y, {%2, %2};\n\t"
+      "add.rn.ftz.f32x2 x, x, y;\n\tmov.b64 {%0, %1}, x;\n\t}"
+      : "+f"(a), "+f"(b)
+      : "f"(s));
+}
+// (a, b) += (c, d)
+__device__ __forceinline__ void acc2(float& a, float& b, float c, float d) {
+  asm("{\n\t.reg .b64 x, y;\n\tmov.b64 x, {%0, %1};\n\tmov.b64 y, {%2, %3};\n\t"
+      "add.rn.ftz.f32x2 x, x, y;\n\tmov.b64 {%0, %1}, x;\n\t}"
+      : "+f"(a), "+f"(b)
+      : "f"(c), "f"(d));
+}
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
 }
 
-// ------------------------------------------------------------------- math
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));

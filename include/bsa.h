@@ -157,8 +157,9 @@ int bsa_forward(const void* Q, const void* K, const void* V,
 /* Bits of the device status word. */
 #define BSA_STATUS_TIMEOUT     0x1u  /* a bounded wait inside the kernel gave up */
 #define BSA_STATUS_BAD_COLUMN  0x2u  /* a column index outside [0, M) was skipped */
-#define BSA_STATUS_BAD_ROW_PTR 0x4u  /* row_ptr[i+1] < row_ptr[i] was seen; the row was treated as empty */
+#define BSA_STATUS_BAD_ROW_PTR 0x4u  /* row_ptr[i] < 0 or row_ptr[i+1] < row_ptr[i] was seen; the row was treated as empty */
 #define BSA_STATUS_BAD_SEQ_LEN 0x8u  /* bsa_decode: a seq_len outside [1, L]; that entry was treated as empty */
+#define BSA_STATUS_INTERNAL    0x10u /* a kernel found its own work plan inconsistent and stopped; a library fault */
 
 /*
  * Content-based top-k block selection (a pattern computed from Q and K on the
@@ -215,6 +216,9 @@ int bsa_topk_pattern(const void* Q, const void* K, int BH, int N, int d, int blo
  * cudaGetSymbolAddress on the first call on each device (the current device
  * at the call), so make that first call before any stream capture on that
  * device.  The call makes no cudaMalloc, cudaFree or other allocating call.
+ * The address is kept for the life of the process: after cudaDeviceReset (or
+ * any reset of the device's primary context) it is stale, so do not call this
+ * entry point again on that device in the same process.
  *
  * Arguments, layouts, results and the other errors are those of
  * bsa_topk_pattern (same kernels, same bits).  A request whose workspace,
