@@ -113,6 +113,10 @@ int launch_fwd(const void* Q, const void* K, const void* V, const int32_t* row_p
   a.W = (a.M + 31) / 32;
   a.num_tiles = BH * a.G;
   a.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+  // The kernel scales masked keys (+-inf) by the scale; a zero scale becomes
+  // the smallest normal float, which leaves every unmasked score at 0 to
+  // within fp32 rounding and sends masked ones to -inf.
+  if (a.scale_log2 == 0.f) a.scale_log2 = 1.17549435e-38f;
   a.causal = causal;
   // stages, control block, the tile-bitmap buffers, and 1024 bytes of alignment slack
   const int smem = C::OFF_CTRL + static_cast<int>(sizeof(pp::Ctrl)) +

@@ -51,6 +51,12 @@ constexpr int kThreads = 32 * kWarps;
 constexpr int kProdWarp = 8;                // producer of slot s is warp kProdWarp + 2 s
 constexpr int kMmaWarp = 9;
 constexpr int kTiRing = 3;                  // tile-info entries per slot
+// One group of 4 probabilities in kPolyEvery is computed by a polynomial on
+// the FMA pipe instead of the MUFU ex2 (0: all by ex2), to relieve the MUFU.
+#ifndef BSA_POLY_EVERY
+#define BSA_POLY_EVERY 4
+#endif
+constexpr int kPolyEvery = BSA_POLY_EVERY;
 
 constexpr int kMaxGrid = 160;               // CTAs per launch (the host caps the grid)
 constexpr int kMaxVirt = kSlots * kMaxGrid; // slots scheduled as workers
@@ -183,7 +189,9 @@ __device__ __forceinline__ long long block_scan(long long v, long long* total, l
 // pattern is shared across b).  Every CTA computes the same plan:
 //  1. total = sum of the tile costs; a tile is heavy when its cost exceeds
 //     thr = total / (2V), half of one slot's share, so there are fewer than
-//     2V heavy tiles.  Heavy tile k (in tile order) goes to slot k mod V.
+//     2V heavy tiles.  When there are at most V, heavy tile k (in tile order)
+//     goes to slot k mod V; when there are more, the costs are too even for
+//     this to pay and every tile is treated as light.
 //  2. The other ("light") tiles, in tile order, are dealt out in rounds of
 //     one tile per slot.
 //  3. When there are at most V heavy tiles, the slots holding one sit out
@@ -221,7 +229,10 @@ __device__ void schedule(const FwdArgs& a, Ctrl* ctl) {
   }
   __syncthreads();  // every thread's heavy groups are written before thread 0 deals them out
   if (tid == 0) {
-    const long long Kh = Kg * nb;  // < 2V <= kMaxHeavyGroups
+    // More heavy tiles than slots means the costs are close to even: plain
+    // rounds then balance better than dealing the "heavy" ones first.
+    if (Kg * nb > V) Kg = 0;
+    const long long Kh = Kg * nb;  // <= V
     const long long n_light = a.num_tiles - Kh;
     long long skip = 0;
     if (Kh > 0 && Kh <= V && n_light > 0 && V - Kh > 0) {
@@ -550,9 +561,12 @@ __device__ void mma_role(const FwdArgs& a, uint8_t* smem, Ctrl* ctl, uint32_t tm
   };
 
   long long idle_since = clock64();
+  int oldest = 0;  // the slot whose pending P V was queued first
   while (!(sl0.done && sl0.pcount == 0 && sl1.done && sl1.pcount == 0)) {
     const int r0 = try_pv(sl0, 0), r1 = try_qk(sl0, 0);
     const int r2 = try_pv(sl1, 1), r3 = try_qk(sl1, 1);
+    if (r0) oldest = 1;
+    if (r2) oldest = 0;
     if (r1 < 0 || r3 < 0) {
       atomicOr(&g_status, BSA_STATUS_INTERNAL);
       ctl->abort.v = 1;
@@ -562,7 +576,16 @@ __device__ void mma_role(const FwdArgs& a, uint8_t* smem, Ctrl* ctl, uint32_t tm
       idle_since = clock64();
     } else {
       if (ctl->abort.v) break;
-      __nanosleep(32);  // leave the issue slots of this sub-partition to the softmax warps
+      // Nothing is ready: sleep in the barrier the issuer most likely waits
+      // for (a slot's P, its softmax warps being the usual hold-up), which
+      // leaves this sub-partition's issue slots to the softmax warps.
+      int ws = oldest;
+      if ((ws == 0 ? sl0.pcount : sl1.pcount) == 0) ws ^= 1;
+      const MmaSlot& w = ws == 0 ? sl0 : sl1;
+      if (w.pcount > 0)
+        mbar_try_wait_hint(&ctl->sb[ws].p_full, w.p_seen & 1, 2000);
+      else
+        __nanosleep(64);
       if (clock64() - idle_since > kWaitLimitCycles) {
         atomicOr(&g_status, BSA_STATUS_TIMEOUT);
         ctl->abort.v = 1;
@@ -658,25 +681,39 @@ __device__ void softmax_role(int s, const FwdArgs& a, Ctrl* ctl, const uint32_t*
           __syncwarp();
           if (lane == 0) mbar_arrive(&B.s_free);
         }
-        float hm = kNegInf;
+        // Row maximum of the scaled scores, taken on the raw scores (their
+        // minimum for a negative scale); on the diagonal block of a causal
+        // tile, keys after the query are first set to the value that scales
+        // to -inf.
+        const bool pos = sl2 > 0.f;
+        const float sentinel = pos ? kNegInf : INFINITY;
+        float hraw = sentinel;
 #pragma unroll
         for (int gi = 0; gi < 2; ++gi) {
           if (!((ho >> gi) & 1u)) continue;
-#pragma unroll
-          for (int c = 0; c < 32; c += 2) mul2(x[gi * 32 + c], x[gi * 32 + c + 1], sl2);
           if ((hd >> gi) & 1u) {               // keys after the query (diagonal block only)
 #pragma unroll
             for (int c = 0; c < 32; ++c)
-              if ((64 * h + gi * 32 + c) % BS > qq) x[gi * 32 + c] = kNegInf;
+              if ((64 * h + gi * 32 + c) % BS > qq) x[gi * 32 + c] = sentinel;
           }
-          float ma = kNegInf, mb = kNegInf;
+          float ma = sentinel, mb = sentinel;
+          if (pos) {
 #pragma unroll
-          for (int c = 0; c < 32; c += 4) {
-            ma = max3f(ma, x[gi * 32 + c], x[gi * 32 + c + 1]);
-            mb = max3f(mb, x[gi * 32 + c + 2], x[gi * 32 + c + 3]);
+            for (int c = 0; c < 32; c += 4) {
+              ma = max3f(ma, x[gi * 32 + c], x[gi * 32 + c + 1]);
+              mb = max3f(mb, x[gi * 32 + c + 2], x[gi * 32 + c + 3]);
+            }
+            hraw = max3f(hraw, ma, mb);
+          } else {
+#pragma unroll
+            for (int c = 0; c < 32; c += 4) {
+              ma = min3f(ma, x[gi * 32 + c], x[gi * 32 + c + 1]);
+              mb = min3f(mb, x[gi * 32 + c + 2], x[gi * 32 + c + 3]);
+            }
+            hraw = min3f(hraw, ma, mb);
           }
-          hm = max3f(hm, ma, mb);
         }
+        const float hm = hraw * sl2;           // -inf when no key of the half is held
         // Lazy rescale: the running maximum moves only when it is exceeded by
         // more than the threshold (P stays <= 2^8 otherwise).
         const bool need = hm > m_used + kRescaleThreshold;
@@ -713,10 +750,17 @@ __device__ void softmax_role(int s, const FwdArgs& a, Ctrl* ctl, const uint32_t*
             for (int c = 0; c < 32; c += 4) {
               float d0 = x[gi * 32 + c], d1 = x[gi * 32 + c + 1];
               float d2 = x[gi * 32 + c + 2], d3 = x[gi * 32 + c + 3];
-              add2(d0, d1, nmu);
-              add2(d2, d3, nmu);
-              const float p0 = ex2_approx(d0), p1 = ex2_approx(d1);
-              const float p2 = ex2_approx(d2), p3 = ex2_approx(d3);
+              fma2(d0, d1, sl2, nmu);              // scaled score minus the maximum
+              fma2(d2, d3, sl2, nmu);
+              float p0, p1, p2, p3;
+              if (kPolyEvery > 0 && (c / 4) % (kPolyEvery > 0 ? kPolyEvery : 1) == kPolyEvery - 1) {
+                exp2_poly2(d0, d1);                // this share of 2^x on the FMA pipe
+                exp2_poly2(d2, d3);
+                p0 = d0; p1 = d1; p2 = d2; p3 = d3;
+              } else {
+                p0 = ex2_approx(d0); p1 = ex2_approx(d1);
+                p2 = ex2_approx(d2); p3 = ex2_approx(d3);
+              }
               acc2(sa, sb, p0, p1);
               acc2(sc, sd, p2, p3);
               pk[gi * 16 + c / 2] = pack_bf16x2(p0, p1);

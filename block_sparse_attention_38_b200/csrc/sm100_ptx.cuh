@@ -47,6 +47,20 @@ __device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
   return done != 0;
 }
 
+// Suspends the thread until the phase of parity `parity` has completed or
+// about `hint_ns` nanoseconds have passed; true when the phase completed.
+__device__ __forceinline__ bool mbar_try_wait_hint(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t done;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(done)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return done != 0;
+}
+
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t done;
   asm volatile(
@@ -387,6 +401,59 @@ __device__ __forceinline__ void acc2(float& a, float& b, float c, float d) {
       "add.rn.ftz.f32x2 x, x, y;\n\tmov.b64 {%0, %1}, x;\n\t}"
       : "+f"(a), "+f"(b)
       : "f"(c), "f"(d));
+}
+// (a, b) = (a, b) * s + c, one rounding per lane
+__device__ __forceinline__ void fma2(float& a, float& b, float s, float c) {
+  asm("{\n\t.reg .b64 x, y, z;\n\tmov.b64 x, {%0, %1};\n\tmov.b64 y, {%2, %2};\n\t"
+      "mov.b64 z, {%3, %3};\n\tfma.rn.ftz.f32x2 x, x, y, z;\n\tmov.b64 {%0, %1}, x;\n\t}"
+      : "+f"(a), "+f"(b)
+      : "f"(s), "f"(c));
+}
+// (a, b) = (a, b) * (xa, xb) + c
+__device__ __forceinline__ void fma2v(float& a, float& b, float xa, float xb, float c) {
+  asm("{\n\t.reg .b64 x, y, z;\n\tmov.b64 x, {%0, %1};\n\tmov.b64 y, {%2, %3};\n\t"
+      "mov.b64 z, {%4, %4};\n\tfma.rn.ftz.f32x2 x, x, y, z;\n\tmov.b64 {%0, %1}, x;\n\t}"
+      : "+f"(a), "+f"(b)
+      : "f"(xa), "f"(xb), "f"(c));
+}
+// (a, b) -= (c, d)
+__device__ __forceinline__ void sub2v(float& a, float& b, float c, float d) {
+  asm("{\n\t.reg .b64 x, y;\n\tmov.b64 x, {%0, %1};\n\tmov.b64 y, {%2, %3};\n\t"
+      "sub.rn.ftz.f32x2 x, x, y;\n\tmov.b64 {%0, %1}, x;\n\t}"
+      : "+f"(a), "+f"(b)
+      : "f"(c), "f"(d));
+}
+
+// 2^a, 2^b on the FMA pipe, for inputs up to 127.  Cody and Waite's range
+// reduction x = n + f, n = rint(x), f in [-1/2, 1/2]; 2^f by the degree-3
+// minimax polynomial of exp2_poly.py (relative error below 7.5e-5); 2^n
+// added to the exponent field.  The rint is the fp32 addition of 1.5 * 2^23,
+// which leaves n in the low mantissa bits of t, so (bits(t) << 23) is n << 23
+// modulo 2^32.  Inputs are clamped at -126.5 so that n >= -126 and the
+// exponent field cannot wrap: anything below comes out as a denormal under
+// 2^-126 (flushed to zero by the ftz arithmetic that follows).
+__device__ __forceinline__ void exp2_poly2(float& a, float& b) {
+  constexpr float kRound = 12582912.f;  // 1.5 * 2^23
+  a = fmaxf(a, -126.5f);
+  b = fmaxf(b, -126.5f);
+  float ta = a, tb = b;
+  add2(ta, tb, kRound);
+  float na = ta, nb = tb;
+  add2(na, nb, -kRound);
+  float fa = a, fb = b;
+  sub2v(fa, fb, na, nb);
+  float pa = 0.0551716685f, pb = 0.0551716685f;
+  fma2v(pa, pb, fa, fb, 0.242611125f);
+  fma2v(pa, pb, fa, fb, 0.693260968f);
+  fma2v(pa, pb, fa, fb, 0.999928057f);
+  a = __uint_as_float(__float_as_uint(pa) + (__float_as_uint(ta) << 23));
+  b = __uint_as_float(__float_as_uint(pb) + (__float_as_uint(tb) << 23));
+}
+
+__device__ __forceinline__ float min3f(float a, float b, float c) {
+  float r;
+  asm("min.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
 }
 __device__ __forceinline__ float max3f(float a, float b, float c) {
   float r;
