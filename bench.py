@@ -43,7 +43,7 @@ if ROOT not in sys.path:
 import workloads  # noqa: E402
 
 METRIC = "block-sparse attn fwd useful TFLOP/s & ms/fwd (1 B200), % of roofline"
-DEFAULT_WORKLOAD = "loglinear_4k"
+DEFAULT_WORKLOAD = "causal_loglinear_32k"
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 KERNEL_DIR = os.path.join(ROOT, "block_sparse_attention_38_b200", "csrc")
@@ -143,7 +143,7 @@ def load_peaks():
 class ClockSampler:
     """nvidia-smi clocks and throttle reasons sampled every 200 ms in the background."""
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
@@ -166,7 +166,11 @@ class ClockSampler:
             self.proc = None
         time.sleep(0.3)
 
-    def stop(self):
+    def stop(self, region=None):
+        """Stop sampling; statistics over the samples taken inside `region`
+        (wall-clock seconds (t0, t1), time.time() based) when given."""
+        import datetime
+
         if self.proc is None:
             return None
         time.sleep(0.25)
@@ -178,19 +182,66 @@ class ClockSampler:
         rows = []
         for line in open(self.path):
             parts = [p.strip() for p in line.split(",")]
-            if len(parts) < 9:
+            if len(parts) < 10:
                 continue
             try:
-                rows.append((float(parts[1]), float(parts[2]), parts[5:9]))
+                ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                rows.append((ts, float(parts[2]), float(parts[3]), float(parts[4]), parts[6:10]))
             except ValueError:
                 continue
         os.unlink(self.path)
         if not rows:
             return None
+        inside = [r for r in rows if region is None or region[0] <= r[0] <= region[1]]
+        use = inside or rows
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for _, _, r in rows for i in range(4) if r[i].lower() == "active"})
-        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": max(r[1] for r in rows),
-                "reasons": reasons, "samples": len(rows)}
+        reasons = sorted({names[i] for r in use for i in range(4) if r[4][i].lower() == "active"})
+        return {"sm_mhz": statistics.median(r[1] for r in use), "sm_max_mhz": max(r[2] for r in rows),
+                "sm_mhz_min": min(r[1] for r in use), "power_w_max": max(r[3] for r in use),
+                "reasons": reasons, "samples": len(rows), "samples_in_timed_region": len(inside)}
+
+
+L2_NOTE = "flushed before every timed step (512 MB write)"
+
+
+def fwd_config(w, nnz: int, world: int, backward: bool = False) -> dict:
+    """The `config` of a forward (or backward) line; both arms print the same one."""
+    c = {"workload": w.name}
+    if backward:
+        c["pass"] = "backward"
+    c.update({"B": w.B, "H": w.H, "N": w.N, "d": w.d, "block_size": w.block_size,
+              "nnz_blocks": int(nnz), "causal": bool(w.causal), "l2": L2_NOTE,
+              "parallelism": f"replicas x{world}"})
+    if w.pattern.kind == workloads.TOPK:
+        c["top_k"] = w.pattern.top_k
+    return c
+
+
+def decode_config(w, tokens_attended: int, world: int) -> dict:
+    """The `config` of a decode line; both arms print the same one."""
+    return {"workload": w.name, "B": w.B, "H": w.H, "L": w.L, "d": w.d,
+            "block_size": w.block_size, "tokens_attended": int(tokens_attended),
+            "append": bool(w.append), "l2": L2_NOTE, "parallelism": f"replicas x{world}"}
+
+
+def soak(step, flush, seconds: float):
+    """Untimed steps (each after its L2 flush) back to back for about
+    `seconds`, right before the timed region: the clock samples then see the
+    GPU under the same load as the timed steps.  Returns (steps, seconds)."""
+    import torch
+
+    if seconds <= 0:
+        return 0, 0.0
+    n = 0
+    t0 = time.time()
+    while True:
+        for _ in range(8):
+            flush.fill_(n & 0xFF)
+            step()
+            n += 1
+        torch.cuda.synchronize()
+        if time.time() - t0 >= seconds:
+            return n, time.time() - t0
 
 
 def cpu_model() -> str:
@@ -283,8 +334,7 @@ def run_reference(args, w, rank, world):
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * statistics.mean(times), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": w_in.name, "B": w_in.B, "H": w_in.H, "N": w_in.N, "d": w_in.d,
-                   "block_size": w_in.block_size},
+        "config": fwd_config(w_in, len(ci), world),
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
                          "sample": f"{rows_done} random query rows of {w.name} over {args.steps} steps"},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -369,6 +419,8 @@ def run_backward(args, w, rank, world, local_rank):
     clocks = ClockSampler(ids[local_rank] if local_rank < len(ids) else str(local_rank))
     if rank == 0:
         clocks.start()
+    region0 = time.time()
+    soak_steps, soak_s = soak(step, flush, args.soak_seconds)
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     if world > 1:
@@ -384,7 +436,7 @@ def run_backward(args, w, rank, world, local_rank):
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
-    clock_info = clocks.stop() if rank == 0 else None
+    clock_info = clocks.stop((region0, time.time())) if rank == 0 else None
     per_step = [s_.elapsed_time(e) for s_, e in zip(starts, ends)]
     total_ms = float(sum(per_step))
     if bsa.backward_status(clear=True) or bsa.device_status(clear=True):
@@ -454,11 +506,7 @@ def run_backward(args, w, rank, world, local_rank):
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
-        "config": {"workload": w.name, "pass": "backward", "B": w.B, "H": w.H, "N": w.N,
-                   "d": w.d, "block_size": w.block_size, "nnz_blocks": int(len(ci_np)),
-                   "causal": bool(w.causal),
-                   "l2": "flushed before every timed step (512 MB write)",
-                   "parallelism": f"replicas x{world}"},
+        "config": fwd_config(w, len(ci_np), world, backward=True),
         "roofline": roof,
         "cpu_baseline": cpu,
         "e2e": {"value": whole_job_tflops(flops, world, e2e_ms), "unit": "TFLOP/s",
@@ -466,6 +514,7 @@ def run_backward(args, w, rank, world, local_rank):
                 "ms_per_step": e2e_ms},
         "gpu_launches": 5 * args.steps,  # D, tile costs, tile orders, dK/dV, dQ
         "clocks": clock_info,
+        "soak": {"steps": soak_steps, "seconds": soak_s},
         "min_ms": min(per_step), "median_ms": statistics.median(per_step),
     }
     print(json.dumps(line), flush=True)
@@ -557,6 +606,8 @@ def run_decode(args, w, rank, world, local_rank):
     clocks = ClockSampler(ids[local_rank] if local_rank < len(ids) else str(local_rank))
     if rank == 0:
         clocks.start()
+    region0 = time.time()
+    soak_steps, soak_s = soak(step, flush, args.soak_seconds)
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     if world > 1:
@@ -572,7 +623,7 @@ def run_decode(args, w, rank, world, local_rank):
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
-    clock_info = clocks.stop() if rank == 0 else None
+    clock_info = clocks.stop((region0, time.time())) if rank == 0 else None
     per_step = [s.elapsed_time(e) for s, e in zip(starts, ends)]
     total_ms = float(sum(per_step))
     status = bsa.decode_status(clear=True)
@@ -650,11 +701,7 @@ def run_decode(args, w, rank, world, local_rank):
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
-        "config": {"workload": w.name, "B": w.B, "H": w.H, "L": w.L, "d": w.d,
-                   "block_size": w.block_size, "tokens_attended": int(tokens.sum()),
-                   "append": bool(w.append),
-                   "l2": "flushed before every timed step (512 MB write)",
-                   "parallelism": f"replicas x{world}"},
+        "config": decode_config(w, tokens.sum(), world),
         "roofline": roof,
         "cpu_baseline": cpu,
         "e2e": {"value": whole_job_tflops(flops, world, e2e_ms), "unit": "TFLOP/s",
@@ -662,6 +709,7 @@ def run_decode(args, w, rank, world, local_rank):
                 "ms_per_step": e2e_ms},
         "gpu_launches": args.steps,
         "clocks": clock_info,
+        "soak": {"steps": soak_steps, "seconds": soak_s},
         "min_ms": min(per_step), "median_ms": statistics.median(per_step),
     }
     print(json.dumps(line), flush=True)
@@ -696,8 +744,7 @@ def run_reference_backward(args, w, rank, world):
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * statistics.mean(times), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": w.name, "pass": "backward", "B": w.B, "H": w.H, "N": w.N,
-                   "d": w.d, "block_size": w.block_size},
+        "config": fwd_config(w, len(ci), world, backward=True),
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
                          "sample": f"{done} random (b, h) backward passes of {w.name} over {args.steps} steps"},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -728,8 +775,7 @@ def run_reference_decode(args, w, rank, world):
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * statistics.mean(times), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": w.name, "B": w.B, "H": w.H, "L": w.L, "d": w.d,
-                   "block_size": w.block_size},
+        "config": decode_config(w, decode_tokens(w, lens_np, rp, ci).sum(), world),
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
                          "sample": f"{done} random (b, h) decode queries of {w.name} over {args.steps} steps"},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -754,6 +800,7 @@ def run_ours(args, w, rank, world, local_rank):
     L = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=dev)
     flush = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
+    fws = torch.empty(bsa.forward_workspace_bytes(w.d), dtype=torch.uint8, device=dev)
     topk = w.pattern.kind == workloads.TOPK
     if topk:
         # The step chooses the pattern on the device from Q and K, then runs
@@ -770,7 +817,7 @@ def run_ours(args, w, rank, world, local_rank):
             if mid is not None:
                 mid.record(stream)
             bsa.forward(q.view(fold), k.view(fold), v.view(fold), rp_s, ci_s, w.block_size,
-                        w.scale, w.causal, out=O.view(fold), lse=L.view(fold[:3]))
+                        w.scale, w.causal, out=O.view(fold), lse=L.view(fold[:3]), workspace=fws)
         launches_per_step = 3  # block means, selection, forward
     else:
         rp_np, ci_np = bsa.build_pattern_from(w.pattern)
@@ -780,7 +827,8 @@ def run_ours(args, w, rank, world, local_rank):
         def step(mid=None):
             if mid is not None:
                 mid.record(stream)
-            bsa.forward(q, k, v, rp, ci, w.block_size, w.scale, w.causal, out=O, lse=L)
+            bsa.forward(q, k, v, rp, ci, w.block_size, w.scale, w.causal, out=O, lse=L,
+                        workspace=fws)
         launches_per_step = 1
     nnz = int(len(ci_np))
     flops = useful_flops(w, nnz)
@@ -796,6 +844,8 @@ def run_ours(args, w, rank, world, local_rank):
     clocks = ClockSampler(ids[local_rank] if local_rank < len(ids) else str(local_rank))
     if rank == 0:
         clocks.start()
+    region0 = time.time()
+    soak_steps, soak_s = soak(step, flush, args.soak_seconds)
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     mids = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
@@ -810,7 +860,7 @@ def run_ours(args, w, rank, world, local_rank):
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
-    clock_info = clocks.stop() if rank == 0 else None
+    clock_info = clocks.stop((region0, time.time())) if rank == 0 else None
     per_step = [s.elapsed_time(e) for s, e in zip(starts, ends)]
     total_ms = float(sum(per_step))
     # the forward kernel alone (for a top-k step, after the selection kernels)
@@ -846,7 +896,7 @@ def run_ours(args, w, rank, world, local_rank):
             rp_s, ci_s = bsa.topk_pattern(qd, kd, w.block_size, w.pattern.top_k, w.causal,
                                           workspace=ws)
             bsa.forward(qd.view(fold), kd.view(fold), vd.view(fold), rp_s, ci_s, w.block_size,
-                        w.scale, w.causal, out=O.view(fold), lse=L.view(fold[:3]))
+                        w.scale, w.causal, out=O.view(fold), lse=L.view(fold[:3]), workspace=fws)
             Oh.copy_(O, non_blocking=True)
             Lh.copy_(L, non_blocking=True)
 
@@ -866,7 +916,7 @@ def run_ours(args, w, rank, world, local_rank):
             s_fw.wait_event(ev_in)
             with torch.cuda.stream(s_fw):
                 bsa.forward(qd[sl], kd[sl], vd[sl], rpd[h0 * w.M:h1 * w.M + 1], cid, w.block_size,
-                            w.scale, w.causal, out=O[sl], lse=L[sl])
+                            w.scale, w.causal, out=O[sl], lse=L[sl], workspace=fws)
                 ev_fw = torch.cuda.Event()
                 ev_fw.record(s_fw)
             s_out.wait_event(ev_fw)
@@ -943,16 +993,14 @@ def run_ours(args, w, rank, world, local_rank):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
-        "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d,
-                   "block_size": w.block_size, "nnz_blocks": nnz, "causal": bool(w.causal),
-                   "l2": "flushed before every timed step (512 MB write)",
-                   "parallelism": f"replicas x{world}"},
+        "config": fwd_config(w, nnz, world),
         "roofline": roof,
         "cpu_baseline": cpu,
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": int(h2d),
                 "d2h_bytes_per_step": int(d2h), "ms_per_step": e2e_ms},
         "gpu_launches": args.steps * launches_per_step,
         "clocks": clock_info,
+        "soak": {"steps": soak_steps, "seconds": soak_s},
         "min_ms": min(per_step), "median_ms": statistics.median(per_step),
     }
     if w.causal:
@@ -961,7 +1009,6 @@ def run_ours(args, w, rank, world, local_rank):
                                                        world, ms)
     if topk:
         # the selection (block means + top-k select kernels) ahead of the forward
-        line["config"]["top_k"] = w.pattern.top_k
         line["selection_ms"] = ms - fwd_ms
     print(json.dumps(line), flush=True)
 
@@ -975,6 +1022,9 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD,
                     choices=list(workloads.WORKLOADS) + list(workloads.DECODE_WORKLOADS))
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--soak-seconds", type=float, default=1.2,
+                    help="untimed steps run back to back right before the timed ones, so that "
+                         "the clock samples cover a loaded GPU")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--backward", action="store_true",
                     help="time the backward pass (dQ, dK, dV) instead of the forward")

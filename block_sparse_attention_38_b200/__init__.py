@@ -85,6 +85,12 @@ def library() -> ctypes.CDLL:
         lib.bsa_forward.argtypes = [vp, vp, vp, vp, vp, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                     ctypes.c_int, ctypes.c_int, ctypes.c_float, ctypes.c_int,
                                     vp, vp, vp]
+        lib.bsa_forward_workspace_bytes.restype = ctypes.c_size_t
+        lib.bsa_forward_workspace_bytes.argtypes = [ctypes.c_int]
+        lib.bsa_forward_ws.restype = ctypes.c_int
+        lib.bsa_forward_ws.argtypes = [vp, vp, vp, vp, vp, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                       ctypes.c_int, ctypes.c_int, ctypes.c_float, ctypes.c_int,
+                                       vp, vp, vp, ctypes.c_size_t, vp]
         lib.bsa_device_status.restype = ctypes.c_int
         lib.bsa_device_status.argtypes = [ctypes.POINTER(ctypes.c_uint32), ctypes.c_int]
         lib.bsa_version.restype = ctypes.c_int
@@ -164,12 +170,21 @@ def validate_pattern(row_ptr: np.ndarray, col_idx: np.ndarray, H: int, M: int,
                                           ci.size, int(H), int(M), int(bool(causal)))
 
 
+def forward_workspace_bytes(d: int) -> int:
+    """Bytes of the chunk workspace bsa_forward_ws can use for head dim d."""
+    return int(library().bsa_forward_workspace_bytes(int(d)))
+
+
 def forward(q, k, v, row_ptr, col_idx, block_size: int, scale: Optional[float] = None,
-            causal: bool = False, out=None, lse=None):
-    """Block-sparse attention forward through bsa_forward on q's device and current stream.
+            causal: bool = False, out=None, lse=None, split: bool = True, workspace=None):
+    """Block-sparse attention forward on q's device and current stream.
 
     q, k, v: CUDA bf16 tensors [B, H, N, d], contiguous.  row_ptr [H*M+1] and
     col_idx [nnz]: CUDA int32 tensors.  Returns (O bf16 [B,H,N,d], LSE fp32 [B,H,N]).
+    With split (the default) the call is bsa_forward_ws, which may cut long
+    tiles into chunks; `workspace` is then a CUDA tensor of at least
+    forward_workspace_bytes(d) bytes (allocated on the current stream when
+    not given).  split=False calls bsa_forward.
     """
     import torch
 
@@ -192,10 +207,23 @@ def forward(q, k, v, row_ptr, col_idx, block_size: int, scale: Optional[float] =
     col_ptr = col_idx.data_ptr() if col_idx.numel() else row_ptr.data_ptr()
     with torch.cuda.device(q.device):
         stream = torch.cuda.current_stream(q.device).cuda_stream
-        rc = lib.bsa_forward(q.data_ptr(), k.data_ptr(), v.data_ptr(), row_ptr.data_ptr(),
-                             col_ptr, B, H, N, d, int(block_size), float(scale),
-                             int(bool(causal)), out.data_ptr(), lse.data_ptr(), stream)
-    _check(rc, "bsa_forward")
+        if not split:
+            rc = lib.bsa_forward(q.data_ptr(), k.data_ptr(), v.data_ptr(), row_ptr.data_ptr(),
+                                 col_ptr, B, H, N, d, int(block_size), float(scale),
+                                 int(bool(causal)), out.data_ptr(), lse.data_ptr(), stream)
+            _check(rc, "bsa_forward")
+            return out, lse
+        if workspace is None:
+            nbytes = int(lib.bsa_forward_workspace_bytes(d))
+            workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=q.device)
+        if not workspace.is_cuda or not workspace.is_contiguous():
+            raise ValueError("workspace must be a contiguous CUDA tensor")
+        rc = lib.bsa_forward_ws(q.data_ptr(), k.data_ptr(), v.data_ptr(), row_ptr.data_ptr(),
+                                col_ptr, B, H, N, d, int(block_size), float(scale),
+                                int(bool(causal)), out.data_ptr(), lse.data_ptr(),
+                                workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                                stream)
+    _check(rc, "bsa_forward_ws")
     return out, lse
 
 

@@ -32,6 +32,14 @@ struct FwdArgs {
   long long num_tiles;
   float scale_log2;       // scale * log2(e)
   int causal;
+  // Chunked tiles (optional): a long tile's key walk is cut into chunks that
+  // run as separate work units; each chunk stores its unnormalised partial
+  // result, and the last chunk to finish merges them.
+  float* part_o;                  // [part_cap][D][128] fp32: O of a chunk before division by l
+  float2* part_ml;                // [part_cap][128]: (running maximum m, log2 units; sum l)
+  unsigned long long* part_cnt;   // [part_cap][4]: per warp, epoch << 8 | chunks arrived
+  int part_cap;                   // chunk slots in the workspace; 0 = no tile is cut
+  unsigned long long epoch;       // distinct for every launch (< 2^56)
 };
 
 struct AbortFlag {
@@ -90,6 +98,23 @@ struct BitIter {
   int W, w;
   uint32_t cur;
   __device__ __forceinline__ BitIter(const uint32_t* b, int W_) : bits(b), W(W_), w(0), cur(b[0]) {}
+  // Passes over the next k set bits (fewer if the map runs out first).
+  __device__ __forceinline__ void skip(int k) {
+    while (k > 0) {
+      if (cur == 0) {
+        if (++w >= W) return;
+        cur = bits[w];
+        continue;
+      }
+      const int c = __popc(cur);
+      if (c <= k) {
+        k -= c;
+        cur = 0;
+      } else {
+        for (; k > 0; --k) cur &= cur - 1;
+      }
+    }
+  }
   __device__ __forceinline__ int next() {
     while (cur == 0) {
       if (++w >= W) return -1;

@@ -4,6 +4,7 @@
 // device status word.  The kernel lives in the headers this file includes;
 // the library's other CUDA translation units are bsa_topk.cu, bsa_decode.cu
 // and bsa_backward.cu.
+#include <atomic>
 #include <mutex>
 
 #include "bsa_common.cuh"
@@ -87,10 +88,20 @@ bool ensure_smem_attr(int dev, int bytes) {
   return true;
 }
 
+// Workspace of the chunked tiles: the count words first (4 per chunk slot,
+// kMaxVirt slots), then per chunk slot its (m, l) pairs and its O columns.
+constexpr size_t kPartHeader = static_cast<size_t>(pp::kMaxVirt) * 4 * 8;
+size_t part_slot_bytes(int d) { return 128 * 8 + 128 * static_cast<size_t>(d) * 4; }
+
+std::atomic<unsigned long long>& launch_epoch() {
+  static std::atomic<unsigned long long> e{1};
+  return e;
+}
+
 template <int BS, int D>
 int launch_fwd(const void* Q, const void* K, const void* V, const int32_t* row_ptr,
                const int32_t* col_idx, int B, int H, int N, float scale, int causal, void* O,
-               float* LSE, cudaStream_t stream) {
+               float* LSE, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
   using C = pp::Cfg<BS, D>;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return BSA_ERR_CUDA;
@@ -118,6 +129,19 @@ int launch_fwd(const void* Q, const void* K, const void* V, const int32_t* row_p
   // within fp32 rounding and sends masked ones to -inf.
   if (a.scale_log2 == 0.f) a.scale_log2 = 1.17549435e-38f;
   a.causal = causal;
+  a.part_o = nullptr;
+  a.part_ml = nullptr;
+  a.part_cnt = nullptr;
+  a.part_cap = 0;
+  a.epoch = launch_epoch().fetch_add(1) & ((1ull << 56) - 1);
+  if (workspace && workspace_bytes >= kPartHeader + part_slot_bytes(D)) {
+    const size_t cap = (workspace_bytes - kPartHeader) / part_slot_bytes(D);
+    a.part_cap = static_cast<int>(cap < static_cast<size_t>(pp::kMaxVirt) ? cap : pp::kMaxVirt);
+    uint8_t* w = static_cast<uint8_t*>(workspace);
+    a.part_cnt = reinterpret_cast<unsigned long long*>(w);
+    a.part_ml = reinterpret_cast<float2*>(w + kPartHeader);
+    a.part_o = reinterpret_cast<float*>(w + kPartHeader + static_cast<size_t>(a.part_cap) * 128 * 8);
+  }
   // stages, control block, the tile-bitmap buffers, and 1024 bytes of alignment slack
   const int smem = C::OFF_CTRL + static_cast<int>(sizeof(pp::Ctrl)) +
                    pp::kSlots * pp::kTiRing * pp::bitmap_words<BS>(a.W) * 4 + 1024;
@@ -133,11 +157,26 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 }  // namespace bsa
 
+extern "C" size_t bsa_forward_workspace_bytes(int d) {
+  using namespace bsa;
+  if (d != 64 && d != 128) return 0;
+  return kPartHeader + static_cast<size_t>(pp::kMaxVirt) * part_slot_bytes(d);
+}
+
 extern "C" int bsa_forward(const void* Q, const void* K, const void* V, const int32_t* row_ptr,
                            const int32_t* col_idx, int B, int H, int N, int d, int block_size,
                            float scale, int causal, void* O, float* LSE, void* stream) {
+  return bsa_forward_ws(Q, K, V, row_ptr, col_idx, B, H, N, d, block_size, scale, causal, O, LSE,
+                        nullptr, 0, stream);
+}
+
+extern "C" int bsa_forward_ws(const void* Q, const void* K, const void* V, const int32_t* row_ptr,
+                              const int32_t* col_idx, int B, int H, int N, int d, int block_size,
+                              float scale, int causal, void* O, float* LSE, void* workspace,
+                              size_t workspace_bytes, void* stream) {
   using namespace bsa;
   if (!Q || !K || !V || !row_ptr || !col_idx || !O || !LSE) return BSA_ERR_INVALID_ARG;
+  if (workspace && !aligned16(workspace)) return BSA_ERR_INVALID_ARG;
   if (B <= 0 || H <= 0 || N <= 0 || d <= 0 || block_size <= 0) return BSA_ERR_INVALID_ARG;
   if (causal != 0 && causal != 1) return BSA_ERR_INVALID_ARG;
   if (!std::isfinite(scale)) return BSA_ERR_INVALID_ARG;
@@ -151,12 +190,12 @@ extern "C" int bsa_forward(const void* Q, const void* K, const void* V, const in
   if (static_cast<long long>(H) * (N / block_size) + 1 > 2147483647LL) return BSA_ERR_UNSUPPORTED;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   switch (block_size * 1000 + d) {
-    case 32064: return launch_fwd<32, 64>(Q, K, V, row_ptr, col_idx, B, H, N, scale, causal, O, LSE, s);
-    case 32128: return launch_fwd<32, 128>(Q, K, V, row_ptr, col_idx, B, H, N, scale, causal, O, LSE, s);
-    case 64064: return launch_fwd<64, 64>(Q, K, V, row_ptr, col_idx, B, H, N, scale, causal, O, LSE, s);
-    case 64128: return launch_fwd<64, 128>(Q, K, V, row_ptr, col_idx, B, H, N, scale, causal, O, LSE, s);
-    case 128064: return launch_fwd<128, 64>(Q, K, V, row_ptr, col_idx, B, H, N, scale, causal, O, LSE, s);
-    case 128128: return launch_fwd<128, 128>(Q, K, V, row_ptr, col_idx, B, H, N, scale, causal, O, LSE, s);
+    case 32064: return launch_fwd<32, 64>(Q, K, V, row_ptr, col_idx, B, H, N, scale, causal, O, LSE, workspace, workspace_bytes, s);
+    case 32128: return launch_fwd<32, 128>(Q, K, V, row_ptr, col_idx, B, H, N, scale, causal, O, LSE, workspace, workspace_bytes, s);
+    case 64064: return launch_fwd<64, 64>(Q, K, V, row_ptr, col_idx, B, H, N, scale, causal, O, LSE, workspace, workspace_bytes, s);
+    case 64128: return launch_fwd<64, 128>(Q, K, V, row_ptr, col_idx, B, H, N, scale, causal, O, LSE, workspace, workspace_bytes, s);
+    case 128064: return launch_fwd<128, 64>(Q, K, V, row_ptr, col_idx, B, H, N, scale, causal, O, LSE, workspace, workspace_bytes, s);
+    case 128128: return launch_fwd<128, 128>(Q, K, V, row_ptr, col_idx, B, H, N, scale, causal, O, LSE, workspace, workspace_bytes, s);
     default: return BSA_ERR_UNSUPPORTED;
   }
 }

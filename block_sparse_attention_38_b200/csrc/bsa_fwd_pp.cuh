@@ -93,19 +93,37 @@ struct Cfg {
   static_assert(QB <= 2 && KS <= 2, "barrier arrays");
 };
 
+constexpr int kMaxChunks = 64;               // chunks one tile may be cut into
+constexpr int kCutShares = 2;                // a tile is cut when it costs more than this many slot shares
+
 // The plan every CTA computes identically (see `schedule`).
 struct Plan {
   long long n_light;                // light tiles in all
-  long long kh;                     // heavy tiles in all
+  long long kt;                     // heavy tiles in all
+  long long kh;                     // heavy work units in all (a cut tile counts once per chunk)
   long long scan[kWarps];
-  int skip;                         // rounds of light tiles a slot holding a heavy tile sits out
+  int skip;                         // rounds of light tiles a slot holding a heavy unit sits out
   int kg;                           // heavy groups per batch element
+  int kc;                           // heavy units per batch element
   int heavy_hg[kMaxHeavyGroups];    // heavy groups of one batch element, in order
+  int heavy_pre[kMaxHeavyGroups + 1];  // heavy units before heavy group j (prefix of chunk counts)
+  int heavy_cs[kMaxHeavyGroups];    // group cost while planning; then steps per chunk
+};
+
+// One work unit: a tile, or one chunk of the key walk of a cut tile.
+struct Unit {
+  long long tile;                   // -1: no more work for this slot
+  int lo;                           // first step of the walk
+  int len;                          // steps at most (the last chunk takes all that remain)
+  int nch;                          // chunks of the tile (1: not cut)
+  int part;                         // workspace slot of this chunk; its tile's chunks are
+                                    // the slots part - c .. part - c + nch - 1
+  int c;                            // chunk index
 };
 
 // One slot's position in the plan (its producer warp advances it).
 struct Cursor {
-  long long heavy[2];               // this slot's heavy tiles
+  long long heavy[2];               // this slot's heavy units
   long long round;                  // next round of light tiles
   long long hp;                     // heavy tiles known to lie before the current light tile
   int n_heavy;
@@ -115,7 +133,8 @@ struct Cursor {
 struct TileInfo {
   long long tile;  // tile index, -1 = no more work for this slot
   int n;           // union size in blocks
-  int pad;
+  int lo, cnt;     // this unit's steps: lo .. lo + cnt - 1 of the walk
+  int nch, part, c;  // see Unit
 };
 
 // The barriers of one slot.
@@ -189,15 +208,19 @@ __device__ __forceinline__ long long block_scan(long long v, long long* total, l
 // pattern is shared across b).  Every CTA computes the same plan:
 //  1. total = sum of the tile costs; a tile is heavy when its cost exceeds
 //     thr = total / (2V), half of one slot's share, so there are fewer than
-//     2V heavy tiles.  When there are at most V, heavy tile k (in tile order)
-//     goes to slot k mod V; when there are more, the costs are too even for
-//     this to pay and every tile is treated as light.
-//  2. The other ("light") tiles, in tile order, are dealt out in rounds of
-//     one tile per slot.
-//  3. When there are at most V heavy tiles, the slots holding one sit out
-//     the first `skip` rounds, skip = average heavy cost / average light cost.
+//     2V heavy tiles.  With more than V of them the costs are too even for
+//     the steps below to pay, and every tile is treated as light.
+//  2. A heavy tile that costs more than kCutShares whole shares (2 thr each)
+//     is cut into chunks of about one share along its key walk ("split long
+//     rows into kv-chunks"), when the caller gave a workspace for the partial
+//     results and the chunks fit in it and in V (else chunks are made longer).
+//  3. The heavy units (uncut heavy tiles and chunks) go first, unit k to slot
+//     k mod V; the light tiles, in tile order, are dealt out in rounds of one
+//     tile per slot, the slots holding a heavy unit sitting out the first
+//     `skip` rounds, skip = average heavy unit cost / average light cost.
 template <int BS>
 __device__ void schedule(const FwdArgs& a, Ctrl* ctl) {
+  constexpr int BPS = 128 / BS;
   Plan& pl = ctl->plan;
   const int tid = threadIdx.x;
   const long long HG = static_cast<long long>(a.H) * a.G;
@@ -225,33 +248,74 @@ __device__ void schedule(const FwdArgs& a, Ctrl* ctl) {
   long long hexcl = block_scan(n_hv, &Kg, pl.scan);
   block_scan(hsum, &Hper, pl.scan);
   for (long long hg = lo; hg < hi && n_hv > 0; ++hg) {
-    if (group_cost<BS>(a, hg) > thr) pl.heavy_hg[hexcl++] = static_cast<int>(hg);
+    const long long cst = group_cost<BS>(a, hg);
+    if (cst > thr) {
+      pl.heavy_hg[hexcl] = static_cast<int>(hg);
+      pl.heavy_cs[hexcl] = static_cast<int>(min(cst, 0x7fffffffLL));
+      ++hexcl;
+    }
   }
   __syncthreads();  // every thread's heavy groups are written before thread 0 deals them out
   if (tid == 0) {
-    // More heavy tiles than slots means the costs are close to even: plain
-    // rounds then balance better than dealing the "heavy" ones first.
     if (Kg * nb > V) Kg = 0;
-    const long long Kh = Kg * nb;  // <= V
-    const long long n_light = a.num_tiles - Kh;
+    // Chunk counts: a group of cost c > kCutShares shares (2 thr each) is cut
+    // into ceil(c / (2 f thr)) chunks, f = 1, 2, 4, ... until all units fit in
+    // V and in the workspace.  (A tile only a little above one share is left
+    // whole: there the cut's own costs, the partial results' round trip and
+    // the chunks' concurrent start, outweigh the balance it buys.)
+    const long long cap = min(V, static_cast<long long>(a.part_cap));
+    const long long cut_above = kCutShares * 2 * thr;
+    long long Kc = Kg;
+    for (long long f = 1; Kg > 0 && cap > 0 && thr > 0; f *= 2) {
+      const long long unit = 2 * f * thr;
+      long long kc = 0;
+      for (long long j = 0; j < Kg; ++j) {
+        const long long cst = pl.heavy_cs[j];
+        kc += cst > cut_above ? min(static_cast<long long>(kMaxChunks), (cst + unit - 1) / unit) : 1;
+      }
+      if (kc * nb <= cap || kc == Kg) {
+        Kc = 0;
+        for (long long j = 0; j < Kg; ++j) {
+          const long long cst = pl.heavy_cs[j];
+          const long long nch =
+              cst > cut_above ? min(static_cast<long long>(kMaxChunks), (cst + unit - 1) / unit) : 1;
+          const long long steps = (cst + BPS - 1) / BPS;  // estimated steps of the walk
+          pl.heavy_pre[j] = static_cast<int>(Kc);
+          pl.heavy_cs[j] = static_cast<int>((steps + nch - 1) / nch);
+          Kc += nch;
+        }
+        break;
+      }
+    }
+    if (Kc == Kg) {  // nothing cut
+      for (long long j = 0; j < Kg; ++j) {
+        pl.heavy_pre[j] = static_cast<int>(j);
+        pl.heavy_cs[j] = 0x7fffffff;
+      }
+    }
+    pl.heavy_pre[Kg] = static_cast<int>(Kc);
+    const long long Kt = Kg * nb;  // heavy tiles
+    const long long Kh = Kc * nb;  // heavy units, <= V
+    const long long n_light = a.num_tiles - Kt;
     long long skip = 0;
-    if (Kh > 0 && Kh <= V && n_light > 0 && V - Kh > 0) {
+    if (Kh > 0 && n_light > 0 && V - Kh > 0) {
       const double heavy_avg = static_cast<double>(Hper * nb) / Kh;
       const double light_avg = static_cast<double>(total - Hper * nb) / n_light;
       skip = static_cast<long long>(heavy_avg / light_avg + 0.5);
       const long long most = n_light / (V - Kh);
       if (skip > most) skip = most;
     }
+    pl.kt = Kt;
     pl.kh = Kh;
     pl.kg = static_cast<int>(Kg);
+    pl.kc = static_cast<int>(Kc);
     pl.n_light = n_light;
     pl.skip = static_cast<int>(skip);
     for (int s = 0; s < kSlots; ++s) {
       Cursor& cu = ctl->cur[s];
       const long long v = static_cast<long long>(kSlots) * blockIdx.x + s;
       int nh = 0;
-      for (long long k = v; k < Kh && nh < 2; k += V)
-        cu.heavy[nh++] = (k / Kg) * HG + pl.heavy_hg[k % Kg];
+      for (long long k = v; k < Kh && nh < 2; k += V) cu.heavy[nh++] = k;
       cu.n_heavy = nh;
       cu.next_heavy = 0;
       cu.round = 0;
@@ -261,15 +325,41 @@ __device__ void schedule(const FwdArgs& a, Ctrl* ctl) {
   __syncthreads();
 }
 
-// Next tile of slot worker v (one builder lane), -1 when none is left: its
-// heavy tiles first, then its light tiles in increasing order.
-__device__ __forceinline__ long long next_tile(const FwdArgs& a, const Plan& pl, Cursor& cu,
-                                               long long v) {
-  if (cu.next_heavy < cu.n_heavy) return cu.heavy[cu.next_heavy++];
+// Heavy unit k of the plan: its tile and its chunk.
+__device__ __forceinline__ Unit heavy_unit(const FwdArgs& a, const Plan& pl, long long k) {
+  const long long HG = static_cast<long long>(a.H) * a.G;
+  const long long b = k / pl.kc;
+  const int r = static_cast<int>(k - b * pl.kc);
+  int lo = 0, hi = pl.kg - 1;  // the group j with heavy_pre[j] <= r < heavy_pre[j + 1]
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (pl.heavy_pre[mid] <= r) lo = mid; else hi = mid - 1;
+  }
+  Unit u;
+  u.tile = b * HG + pl.heavy_hg[lo];
+  u.nch = pl.heavy_pre[lo + 1] - pl.heavy_pre[lo];
+  u.c = r - pl.heavy_pre[lo];
+  u.lo = u.nch > 1 ? u.c * pl.heavy_cs[lo] : 0;
+  u.len = u.c < u.nch - 1 ? pl.heavy_cs[lo] : 0x7fffffff;
+  u.part = static_cast<int>(k);
+  return u;
+}
+
+// Next unit of slot worker v (one builder lane), tile -1 when none is left:
+// its heavy units first, then its light tiles in increasing order.
+__device__ __forceinline__ Unit next_unit(const FwdArgs& a, const Plan& pl, Cursor& cu, long long v) {
+  if (cu.next_heavy < cu.n_heavy) return heavy_unit(a, pl, cu.heavy[cu.next_heavy++]);
+  Unit u;
+  u.tile = -1;
+  u.lo = 0;
+  u.len = 0x7fffffff;
+  u.nch = 1;
+  u.part = 0;
+  u.c = 0;
   const long long V = static_cast<long long>(kSlots) * gridDim.x;
   const long long Kh = pl.kh;
-  const bool skipping = pl.skip > 0;             // at most V heavy tiles, slots 0..Kh-1 hold one
-  const long long others = V - Kh;               // slots without a heavy tile
+  const bool skipping = pl.skip > 0;             // slots 0 .. Kh-1 hold a heavy unit
+  const long long others = V - Kh;               // slots without one
   const long long k = cu.round++;
   long long i;                                   // index among the light tiles
   if (!skipping) {
@@ -284,16 +374,17 @@ __device__ __forceinline__ long long next_tile(const FwdArgs& a, const Plan& pl,
   } else {
     i = static_cast<long long>(pl.skip) * others + (k - pl.skip) * V + v;
   }
-  if (i >= pl.n_light) return -1;
+  if (i >= pl.n_light) return u;
   // Light tile i is tile i + (heavy tiles before it); the heavy tiles are in
   // increasing tile order and i only grows, so the count is kept across calls.
   const long long HG = static_cast<long long>(a.H) * a.G;
   long long t = i + cu.hp;
-  while (cu.hp < Kh && (cu.hp / pl.kg) * HG + pl.heavy_hg[cu.hp % pl.kg] <= t) {
+  while (cu.hp < pl.kt && (cu.hp / pl.kg) * HG + pl.heavy_hg[cu.hp % pl.kg] <= t) {
     ++cu.hp;
     t = i + cu.hp;
   }
-  return t;
+  u.tile = t;
+  return u;
 }
 
 // ---------------------------------------------------------- producer warps
@@ -313,7 +404,8 @@ __device__ void produce_role(int s, const CUtensorMap* tmQ, const CUtensorMap* t
   const long long v = static_cast<long long>(kSlots) * blockIdx.x + s;
   SlotBars& B = ctl->sb[s];
   uint32_t q_loads = 0, k_loads = 0, v_loads = 0;
-  long long peeked = -2;  // lane 0: the slot's next tile, once looked up
+  Unit peeked;            // lane 0: the slot's next unit, once looked up
+  bool have_peek = false;
   bool ok = true;
   if (lane == 0) {
     prefetch_tensormap(tmQ);
@@ -323,15 +415,21 @@ __device__ void produce_role(int s, const CUtensorMap* tmQ, const CUtensorMap* t
   for (int t = 0;; ++t) {
     const int buf = t % kTiRing;
     int w_ok = 1;
-    long long tile = -1;
+    Unit u;
+    u.tile = -1;
     if (lane == 0) {
       w_ok = wait_bounded(&B.t_empty[buf], ((t / kTiRing) & 1) ^ 1, &ctl->abort);
       if (w_ok) {
-        tile = peeked == -2 ? next_tile(a, ctl->plan, ctl->cur[s], v) : peeked;
-        peeked = tile >= 0 ? next_tile(a, ctl->plan, ctl->cur[s], v) : -1;
-        if (peeked >= 0) {  // the next tile's Q into L2
-          const long long pbh = peeked / a.G;
-          const int pg = static_cast<int>(peeked - pbh * a.G);
+        u = have_peek ? peeked : next_unit(a, ctl->plan, ctl->cur[s], v);
+        if (u.tile >= 0) {
+          peeked = next_unit(a, ctl->plan, ctl->cur[s], v);
+        } else {
+          peeked.tile = -1;
+        }
+        have_peek = true;
+        if (peeked.tile >= 0) {  // the next unit's Q into L2
+          const long long pbh = peeked.tile / a.G;
+          const int pg = static_cast<int>(peeked.tile - pbh * a.G);
 #pragma unroll
           for (int ka = 0; ka < C::KATOMS; ++ka)
             tma_prefetch_3d(tmQ, ka * 64, pg * C::TM, static_cast<int>(pbh));
@@ -339,7 +437,7 @@ __device__ void produce_role(int s, const CUtensorMap* tmQ, const CUtensorMap* t
       }
     }
     if (!__shfl_sync(0xffffffffu, w_ok, 0)) { ok = false; break; }
-    tile = __shfl_sync(0xffffffffu, tile, 0);
+    const long long tile = __shfl_sync(0xffffffffu, u.tile, 0);
     uint32_t* bm = bitmaps + (s * kTiRing + buf) * BMW;
     int n = 0;
     long long bh = 0;
@@ -374,6 +472,19 @@ __device__ void produce_role(int s, const CUtensorMap* tmQ, const CUtensorMap* t
       __syncwarp();
       n = union_count(bm + C::R * W, W);
     }
+    // This unit's part of the walk.
+    const int all_steps = (n + C::BPS - 1) / C::BPS;
+    int lo = 0, cnt = 0;
+    if (lane == 0 && tile >= 0) {
+      lo = min(u.lo, all_steps);
+      cnt = min(u.len, all_steps - lo);
+      TileInfo& ti = ctl->info[s][buf];
+      ti.lo = lo;
+      ti.cnt = cnt;
+      ti.nch = u.nch;
+      ti.part = u.part;
+      ti.c = u.c;
+    }
     if (lane == 0) {
       ctl->info[s][buf].tile = tile;
       ctl->info[s][buf].n = n;
@@ -382,7 +493,7 @@ __device__ void produce_role(int s, const CUtensorMap* tmQ, const CUtensorMap* t
     if (lane == 0) mbar_arrive(&B.t_full[buf]);
     if (tile < 0) break;
     if (lane == 0) {
-      if (n > 0) {
+      if (cnt > 0) {
         const uint32_t qb = q_loads % C::QB;
         ok = wait_bounded(&B.q_empty[qb], ((q_loads / C::QB) & 1) ^ 1, &ctl->abort);
         if (ok) {
@@ -394,8 +505,8 @@ __device__ void produce_role(int s, const CUtensorMap* tmQ, const CUtensorMap* t
           ++q_loads;
         }
         BitIter it(bm + C::R * W, W);
-        const int steps = (n + C::BPS - 1) / C::BPS;
-        for (int j = 0; ok && j < steps; ++j) {
+        it.skip(lo * C::BPS);
+        for (int j = 0; ok && j < cnt; ++j) {
           int row0[C::BPS];  // first token of each block of the step; N (out of range) pads
 #pragma unroll
           for (int b = 0; b < C::BPS; ++b) {
@@ -495,13 +606,14 @@ __device__ void mma_role(const FwdArgs& a, uint8_t* smem, Ctrl* ctl, uint32_t tm
         st.done = true;
         return 0;
       }
-      if (tile >= a.num_tiles || n > a.M) return -1;  // never for a consistent schedule
-      if (n == 0) {
+      const int cnt = ctl->info[s][buf].cnt;
+      if (tile >= a.num_tiles || n > a.M || cnt < 0 || cnt > n) return -1;  // never for a consistent schedule
+      if (cnt == 0) {
         mbar_arrive(&B.t_empty[buf]);
         ++st.t;
         return 1;
       }
-      st.qsteps = (n + C::BPS - 1) / C::BPS;
+      st.qsteps = cnt;
       st.qj = 0;
     }
     if (!C::SEP_P && st.pcount > 0) return 0;  // P lives in S: its P V goes first
@@ -598,6 +710,99 @@ __device__ void mma_role(const FwdArgs& a, uint8_t* smem, Ctrl* ctl, uint32_t tm
   wait_drain(&ctl->final_bar, 0);
 }
 
+// ------------------------------------------------------------ chunk merge
+// Arrival of one warp's chunk at its tile's count word (epoch << 8 | count):
+// a word from an earlier launch counts as zero.  Returns the count with this
+// arrival included.
+__device__ __forceinline__ int chunk_arrive(unsigned long long* word, unsigned long long epoch) {
+  unsigned long long old = *reinterpret_cast<volatile unsigned long long*>(word);
+  for (;;) {
+    const unsigned long long nv = (old >> 8) == epoch ? old + 1ull : (epoch << 8) | 1ull;
+    const unsigned long long seen = atomicCAS(word, old, nv);
+    if (seen == old) return static_cast<int>(nv & 0xffull);
+    old = seen;
+  }
+}
+
+// Epilogue of one chunk of a cut tile, per warp (its 32 query rows): store
+// the chunk's O (still multiplied by l) and its (m, l); the warp whose arrival
+// completes the count of its quadrant merges the tile's chunks in chunk
+// order, O = sum_c 2^(m_c - M) O_c / L and LSE = (M + log2 L) ln 2 with
+// M = max_c m_c and L = sum_c 2^(m_c - M) l_c over the chunks holding keys
+// of the row -- the same softmax over the union of the chunks' keys ("Block
+// Sparse Attention with Log-Linear Complexity", section 3.3).  Every chunk,
+// its own included, is read back from the workspace, so the result does not
+// depend on which chunk finishes last.
+template <int D>
+__device__ __forceinline__ void chunk_epilogue(const FwdArgs& a, const TileInfo& ti, uint32_t t_o,
+                                               float m_used, float l, int row, int wq, bool row_ok,
+                                               uint4* orow, float* lse) {
+  const int lane = threadIdx.x & 31;
+  const int part = ti.part, base = ti.part - ti.c, nch = ti.nch;
+  const bool have_o = ti.cnt > 0;  // uniform over the warp
+  float* po = a.part_o + static_cast<long long>(part) * D * 128 + row;
+#pragma unroll 1
+  for (int c0 = 0; c0 < D; c0 += 32) {
+    uint32_t w[32];
+    if (have_o) {
+      __syncwarp();
+      tmem_ld32_wait(t_o + c0, w);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) w[i] = 0u;
+    }
+#pragma unroll
+    for (int i = 0; i < 32; ++i) __stcg(po + (c0 + i) * 128, __uint_as_float(w[i]));
+  }
+  __stcg(a.part_ml + static_cast<long long>(part) * 128 + row, make_float2(m_used, l));
+  __threadfence();
+  __syncwarp();
+  int last = 0;
+  if (lane == 0) last = chunk_arrive(a.part_cnt + static_cast<long long>(base) * 4 + wq, a.epoch) == nch;
+  if (!__shfl_sync(0xffffffffu, last, 0)) return;
+  __threadfence();
+
+  const float2* ml0 = a.part_ml + static_cast<long long>(base) * 128 + row;
+  float M = -INFINITY;
+  for (int cc = 0; cc < nch; ++cc) {
+    const float2 ml = __ldcg(ml0 + cc * 128);
+    if (ml.y > 0.f) M = fmaxf(M, ml.x);
+  }
+  float L = 0.f;
+  for (int cc = 0; cc < nch; ++cc) {
+    const float2 ml = __ldcg(ml0 + cc * 128);
+    if (ml.y > 0.f) L += ml.y * ex2_approx(ml.x - M);
+  }
+  const float inv = L > 0.f ? 1.f / L : 0.f;
+  const float* pb = a.part_o + static_cast<long long>(base) * D * 128 + row;
+#pragma unroll 1
+  for (int c0 = 0; c0 < D; c0 += 32) {
+    float acc[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) acc[i] = 0.f;
+#pragma unroll 1
+    for (int cc = 0; cc < nch; ++cc) {
+      const float2 ml = __ldcg(ml0 + cc * 128);
+      const float wt = ml.y > 0.f ? ex2_approx(ml.x - M) * inv : 0.f;
+      const float* pc = pb + static_cast<long long>(cc) * D * 128 + c0 * 128;
+#pragma unroll
+      for (int i = 0; i < 32; ++i) acc[i] = fmaf(wt, __ldcg(pc + i * 128), acc[i]);
+    }
+    if (row_ok) {
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        uint4 v;
+        v.x = pack_bf16x2(acc[q * 8 + 0], acc[q * 8 + 1]);
+        v.y = pack_bf16x2(acc[q * 8 + 2], acc[q * 8 + 3]);
+        v.z = pack_bf16x2(acc[q * 8 + 4], acc[q * 8 + 5]);
+        v.w = pack_bf16x2(acc[q * 8 + 6], acc[q * 8 + 7]);
+        orow[c0 / 8 + q] = v;
+      }
+    }
+  }
+  if (row_ok) *lse = L > 0.f ? (M + __log2f(L)) * 0.69314718055994531f : -INFINITY;
+}
+
 // ------------------------------------------------------- softmax warpgroups
 // Warpgroup s: thread i owns query row i of slot s's tile.  A step is taken
 // in two halves of 64 score columns: load the blocks the row holds, scale,
@@ -633,7 +838,9 @@ __device__ void softmax_role(int s, const FwdArgs& a, Ctrl* ctl, const uint32_t*
     const long long tile = ctl->info[s][buf].tile;
     const int n = ctl->info[s][buf].n;
     if (tile < 0) return;
-    if (tile >= a.num_tiles || n > a.M) {     // never for a consistent schedule
+    const TileInfo& ti = ctl->info[s][buf];  // in shared memory until the t_empty arrival
+    if (tile >= a.num_tiles || n > a.M || ti.cnt < 0 || ti.cnt > n ||
+        (ti.nch > 1 && (ti.part < ti.c || ti.part - ti.c + ti.nch > a.part_cap))) {  // never for a consistent schedule
       if (lane == 0) {
         atomicOr(&g_status, BSA_STATUS_INTERNAL);
         ctl->abort.v = 1;
@@ -646,9 +853,9 @@ __device__ void softmax_role(int s, const FwdArgs& a, Ctrl* ctl, const uint32_t*
 
     float m_used = kNegInf;  // running maximum, log2 units of the scaled score
     float l = 0.f;           // running sum of 2^(x - m_used)
-    const int steps = (n + C::BPS - 1) / C::BPS;
     BitIter it(bm + C::R * W, W);
-    for (int j = 0; j < steps; ++j) {
+    it.skip(ti.lo * C::BPS);
+    for (int j = 0; j < ti.cnt; ++j) {
       // 32-column groups of this step whose block this row holds, and those
       // of its diagonal block (both uniform over the warp).
       uint32_t own = 0, diag = 0;
@@ -805,16 +1012,23 @@ __device__ void softmax_role(int s, const FwdArgs& a, Ctrl* ctl, const uint32_t*
     const long long bh = tile / a.G;
     const long long qtok = (tile - bh * a.G) * C::TM + row;
     uint4* orow = reinterpret_cast<uint4*>(a.O + (bh * a.N + qtok) * D);
-    if (n > 0) {
+    if (ti.cnt > 0) {
       if (!warp_wait(&B.o_full, o_seen & 1, &ctl->abort)) return;
       ++o_seen;
       tc_fence_after();
+    }
+    if (ti.nch > 1) {
+      chunk_epilogue<D>(a, ti, t_o, m_used, l, row, wq, row_ok, orow, a.LSE + bh * a.N + qtok);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&B.t_empty[buf]);
+      continue;
     }
     const float inv = l > 0.f ? 1.f / l : 0.f;
 #pragma unroll 1
     for (int c0 = 0; c0 < D; c0 += 32) {
       uint32_t w[32];
-      if (n > 0) {
+      if (ti.cnt > 0) {
         __syncwarp();
         tmem_ld32_wait(t_o + c0, w);
       } else {

@@ -154,6 +154,34 @@ int bsa_forward(const void* Q, const void* K, const void* V,
                 int B, int H, int N, int d, int block_size, float scale, int causal,
                 void* O, float* LSE, void* stream);
 
+/*
+ * bsa_forward_ws -- bsa_forward with a workspace for chunked tiles.
+ *
+ * The kernel's unit of work is a tile of 128 query rows walking the union of
+ * its block rows' columns.  When one tile's walk is longer than an even share
+ * of the whole launch per tile slot (a global row, a long causal row), its
+ * walk is cut into chunks that run as separate units; each chunk leaves its
+ * unnormalised O and its (max, sum) statistics in the workspace and the last
+ * chunk of the tile to finish merges them, weighting chunk c by
+ * exp(m_c - max_c m_c) ("split long rows into kv-chunks"; the merged softmax
+ * is the one of section 3.3 of "Block Sparse Attention with Log-Linear
+ * Complexity" over the union of the chunks' keys).  The result is the same
+ * function as bsa_forward's, up to fp32 rounding.
+ *
+ * Arguments as bsa_forward, plus workspace: caller-owned device memory,
+ * 16-byte aligned, of up to bsa_forward_workspace_bytes(d) bytes (a smaller
+ * one allows fewer chunks; below one chunk, or NULL, no tile is cut, which is
+ * bsa_forward).  Its contents need not be initialised and are overwritten;
+ * one workspace must not serve two launches that may run at the same time.
+ * Nothing is allocated and nothing synchronised.  Errors as bsa_forward;
+ * BSA_ERR_INVALID_ARG also for a misaligned workspace.
+ */
+size_t bsa_forward_workspace_bytes(int d);  /* 0 for an unsupported d */
+int bsa_forward_ws(const void* Q, const void* K, const void* V,
+                   const int32_t* row_ptr, const int32_t* col_idx,
+                   int B, int H, int N, int d, int block_size, float scale, int causal,
+                   void* O, float* LSE, void* workspace, size_t workspace_bytes, void* stream);
+
 /* Bits of the device status word. */
 #define BSA_STATUS_TIMEOUT     0x1u  /* a bounded wait inside the kernel gave up */
 #define BSA_STATUS_BAD_COLUMN  0x2u  /* a column index outside [0, M) was skipped */
