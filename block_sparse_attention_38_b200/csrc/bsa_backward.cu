@@ -176,39 +176,82 @@ __global__ void tile_cost_kernel(const int32_t* __restrict__ ptr_a, const int32_
 // when the heaviest tile costs more than twice the mean, or when the launch
 // is a few waves (T < few_waves tiles) and the last, partial wave should hold
 // the lightest tiles; else in index order, which keeps the tiles of one
-// (b, h) together and their K/V shared in L2.
-__global__ void __launch_bounds__(1024) tile_order_kernel(const int* __restrict__ cost, long long T,
-                                                          long long few_waves,
-                                                          int* __restrict__ order) {
+// (b, h) together and their K/V shared in L2.  Launched with kOrderThreads
+// threads per block: each thread takes kCostBins / kOrderThreads adjacent
+// bins, and the bin offsets come from one block-wide scan.
+constexpr int kOrderThreads = 1024;
+
+__global__ void __launch_bounds__(kOrderThreads) tile_order_kernel(const int* __restrict__ cost,
+                                                                   long long T, long long few_waves,
+                                                                   int* __restrict__ order) {
+  constexpr int kPer = kCostBins / kOrderThreads;  // bins per thread
+  constexpr int kOrderWarps = kOrderThreads / 32;
+  static_assert(kCostBins % kOrderThreads == 0, "bins split evenly over the threads");
   __shared__ int hist[kCostBins];
+  __shared__ long long warp_total[kOrderWarps];
+  __shared__ int warp_count[kOrderWarps], warp_top[kOrderWarps];
   __shared__ int sorted;
   const int* c = cost + blockIdx.x * T;
   int* o = order + blockIdx.x * T;
-  for (int b = threadIdx.x; b < kCostBins; b += blockDim.x) hist[b] = 0;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  for (int b = tid; b < kCostBins; b += kOrderThreads) hist[b] = 0;
   __syncthreads();
-  for (long long t = threadIdx.x; t < T; t += blockDim.x) atomicAdd(&hist[c[t]], 1);
+  for (long long t = tid; t < T; t += kOrderThreads) atomicAdd(&hist[c[t]], 1);
   __syncthreads();
-  if (threadIdx.x == 0) {
-    long long total = 0;
-    int top = 0;
-    for (int b = 0; b < kCostBins; ++b) {
-      total += static_cast<long long>(b) * hist[b];
-      if (hist[b] > 0) top = b;
+  // This thread's bins, heaviest first: kCostBins-1 - (tid*kPer + i).
+  int cnt[kPer];
+  int n = 0, top = 0;
+  long long total = 0;
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) {
+    const int b = kCostBins - 1 - (tid * kPer + i);
+    cnt[i] = hist[b];
+    n += cnt[i];
+    total += static_cast<long long>(b) * cnt[i];
+    if (cnt[i] > 0) top = max(top, b);
+  }
+  int incl = n;  // inclusive scan of the counts in thread order (descending bins)
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int x = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += x;
+  }
+  long long wt = total;
+  int wtop = top;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    wt += __shfl_xor_sync(0xffffffffu, wt, off);
+    wtop = max(wtop, __shfl_xor_sync(0xffffffffu, wtop, off));
+  }
+  if (lane == 31) warp_count[warp] = incl;
+  if (lane == 0) {
+    warp_total[warp] = wt;
+    warp_top[warp] = wtop;
+  }
+  __syncthreads();
+  int run = incl - n;
+  for (int w = 0; w < warp; ++w) run += warp_count[w];
+  if (tid == 0) {
+    long long all = 0;
+    int heaviest = 0;
+    for (int w = 0; w < kOrderWarps; ++w) {
+      all += warp_total[w];
+      heaviest = max(heaviest, warp_top[w]);
     }
-    sorted = static_cast<long long>(top) * T > 2 * total || T < few_waves;
-    int run = 0;  // exclusive offsets, heaviest bin first
-    for (int b = kCostBins - 1; b >= 0; --b) {
-      const int n = hist[b];
-      hist[b] = run;
-      run += n;
-    }
+    sorted = static_cast<long long>(heaviest) * T > 2 * all || T < few_waves;
+  }
+  __syncthreads();  // every thread has read its counts before the offsets overwrite them
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) {
+    hist[kCostBins - 1 - (tid * kPer + i)] = run;  // exclusive offset, heaviest bin first
+    run += cnt[i];
   }
   __syncthreads();
   if (sorted) {
-    for (long long t = threadIdx.x; t < T; t += blockDim.x)
+    for (long long t = tid; t < T; t += kOrderThreads)
       o[atomicAdd(&hist[c[t]], 1)] = static_cast<int>(t);
   } else {
-    for (long long t = threadIdx.x; t < T; t += blockDim.x) o[t] = static_cast<int>(t);
+    for (long long t = tid; t < T; t += kOrderThreads) o[t] = static_cast<int>(t);
   }
 }
 
@@ -790,7 +833,7 @@ int launch(const void* Q, const void* K, const void* V, const void* dO, Args a, 
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess)
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  tile_order_kernel<<<2, 1024, 0, s>>>(cost, T, 8LL * sms, order);
+  tile_order_kernel<<<2, kOrderThreads, 0, s>>>(cost, T, 8LL * sms, order);
   if (cudaGetLastError() != cudaSuccess) return BSA_ERR_CUDA;
   Args kv = a;
   kv.ptr = col_ptr;

@@ -85,3 +85,65 @@ def test_tiny_loglinear_workload():
     w = workloads.WORKLOADS["tiny_loglinear"]
     rp, ci = bsa.build_pattern_from(w.pattern)
     _run(w.B, w.H, w.N, w.d, w.block_size, rp, ci, w.causal, seed=w.seed)
+
+
+def _check_grads(got_list, ref_list, what):
+    for name, got, want in zip(("dQ", "dK", "dV"), got_list, ref_list):
+        g_ = np.asarray(got, dtype=np.float64)
+        assert np.isfinite(g_).all(), (what, name)
+        err = np.abs(g_ - want)
+        scale_max = max(np.abs(want).max(), 1e-6)
+        scale_mean = max(np.abs(want).mean(), 1e-6)
+        assert err.max() <= 2e-2 * scale_max, (what, name, err.max(), scale_max)
+        assert err.mean() <= 1e-2 * scale_mean, (what, name, err.mean(), scale_mean)
+
+
+@pytest.mark.parametrize("name,branch", [("bernoulli_4k", "index"), ("local_global_8k", "sorted")])
+def test_full_size_backward(name, branch):
+    """The full workload in one backward launch (the bench's), compared on
+    sampled (b, h) with the oracle.  bernoulli_4k (4096 tiles of even cost)
+    runs its tiles in index order; local_global_8k (tiles of the global rows
+    and columns far above the mean) in heavy-first order: the tile orders in
+    the workspace show which branch ran."""
+    w = workloads.WORKLOADS[name]
+    B, H, N, d, bs = w.B, w.H, w.N, w.d, w.block_size
+    q, k, v = workloads.make_qkv(w)
+    g = torch.Generator().manual_seed(w.seed + 77)
+    do = torch.randn(q.shape, generator=g).to(torch.bfloat16)
+    rp, ci = bsa.build_pattern_from(w.pattern)
+    cp, ri = bsa.transpose_pattern(rp, ci, H, w.M)
+    dev = lambda x: torch.from_numpy(np.ascontiguousarray(x, dtype=np.int32)).to(DEV)  # noqa: E731
+    rpd, cid, cpd, rid = dev(rp), dev(ci), dev(cp), dev(ri)
+    qd, kd, vd, dod = (t.to(DEV) for t in (q, k, v, do))
+    O, L = bsa.forward(qd, kd, vd, rpd, cid, bs, w.scale, w.causal)
+    nbytes = bsa.library().bsa_backward_workspace_bytes(B, H, N)
+    ws = torch.empty(nbytes // 4, dtype=torch.float32, device=DEV)
+    dq, dk, dv = bsa.backward(qd, kd, vd, O, dod, L, rpd, cid, cpd, rid, bs, w.scale, w.causal,
+                              workspace=ws)
+    torch.cuda.synchronize()
+    assert bsa.device_status(clear=True) == 0
+    assert bsa.backward_status(clear=True) == 0
+
+    rows, T = B * H * N, B * H * (N // 128)
+    words = ws.view(torch.int32).cpu().numpy()
+    cost = words[rows:rows + 2 * T]
+    order = words[rows + 2 * T:rows + 4 * T]
+    for half in range(2):
+        o = order[half * T:(half + 1) * T]
+        c = cost[half * T:(half + 1) * T]
+        assert np.array_equal(np.sort(o), np.arange(T))
+        if branch == "index":
+            assert np.array_equal(o, np.arange(T))
+        else:
+            assert np.all(np.diff(c[o]) <= 0) and not np.array_equal(o, np.arange(T))
+
+    rng = np.random.default_rng(0)
+    pairs = {(0, 0), (B - 1, H - 1), (int(rng.integers(B)), int(rng.integers(H)))}
+    got = [t.float().cpu().numpy() for t in (dq, dk, dv)]
+    M = w.M
+    for b, h in sorted(pairs):
+        rph = (rp[h * M:(h + 1) * M + 1] - rp[h * M]).astype(np.int32)
+        cih = ci[rp[h * M]:rp[(h + 1) * M]]
+        sl = (slice(b, b + 1), slice(h, h + 1))
+        ref = obw.backward(q[sl], k[sl], v[sl], do[sl], rph, cih, bs, w.scale, w.causal)
+        _check_grads([x[b, h] for x in got], [r[0, 0] for r in ref], f"{name} b{b} h{h}")
