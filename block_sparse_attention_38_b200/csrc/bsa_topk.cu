@@ -13,10 +13,14 @@
 //                  means are stored transposed, [bh][c][block], so that the
 //                  threads of the selection (one per candidate block) read
 //                  consecutive addresses for each c
-//   select_kernel  one CTA per (bh, block row): scores of the M candidate
-//                  blocks into shared memory, a bitonic sort on (score
-//                  descending, column ascending), then the chosen columns
-//                  written in ascending order at the row's fixed CSR offset
+//   select_warp_kernel  (M <= 1024) one warp per (bh, block row): the
+//                  candidates' scores, a bitonic sort and the selection, all
+//                  in registers (see below)
+//   select_kernel  (larger M) one CTA per (bh, block row): scores of the M
+//                  candidate blocks into shared memory, a bitonic sort on
+//                  (score descending, column ascending), then the chosen
+//                  columns written in ascending order at the row's fixed CSR
+//                  offset
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -159,6 +163,145 @@ __global__ void __launch_bounds__(kSelectThreads)
   }
 }
 
+// One warp per (bh, block row) for M <= 1024: lane l takes the candidates
+// j = l + 32e (e < E, E = Mp / 32), scores them with the same fixed-order fp64
+// chain as select_kernel (E independent chains per lane), sorts the Mp
+// (score, column) pairs with a bitonic network held in registers (pairs 32
+// or more apart swap inside a lane, closer ones between lanes by shuffle),
+// marks the first `keep` columns and the diagonal in a per-warp bitmap, and
+// writes the marked columns in ascending order.
+constexpr int kWarpRowsPerCta = 8;
+
+template <int E>
+__global__ void __launch_bounds__(32 * kWarpRowsPerCta)
+    select_warp_kernel(const double* __restrict__ qm, const double* __restrict__ kmT, int M, int d,
+                       int top_k, int causal, int32_t* __restrict__ row_ptr,
+                       int32_t* __restrict__ col_idx, long long num_rows) {
+  __shared__ uint32_t marks[kWarpRowsPerCta][32];
+  const int lane = threadIdx.x & 31, wl = threadIdx.x >> 5;
+  const long long r = static_cast<long long>(blockIdx.x) * kWarpRowsPerCta + wl;  // bh * M + i
+  if (r >= num_rows) return;
+  const long long bh = r / M;
+  const int i = static_cast<int>(r - bh * M);
+  const double* qrow = qm + r * d;
+  const double* kbase = kmT + bh * static_cast<long long>(M) * d;
+
+  double sc[E];
+  int col[E];
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    col[e] = lane + 32 * e;
+    sc[e] = 0.0;
+  }
+  // U columns c per round: all their loads are issued before the first of
+  // their products, so one round costs one memory latency; the sums still
+  // run over c in ascending order.
+  constexpr int U = 64 / E;  // 64 loads in flight per lane and round
+  for (int c0 = 0; c0 < d; c0 += U) {
+    double qv[U], kv[U][E];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int c = c0 + u;
+      qv[u] = c < d ? __ldg(qrow + c) : 0.0;
+      const double* kc = kbase + static_cast<long long>(c) * M;
+#pragma unroll
+      for (int e = 0; e < E; ++e) kv[u][e] = (c < d && col[e] < M) ? __ldg(kc + col[e]) : 0.0;
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      if (c0 + u >= d) break;
+#pragma unroll
+      for (int e = 0; e < E; ++e)
+        if (col[e] < M) sc[e] = __dadd_rn(sc[e], __dmul_rn(qv[u], kv[u][e]));
+    }
+  }
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    const int j = col[e];
+    if (j >= M || j == i || (causal && j > i)) sc[e] = -INFINITY;  // not a candidate: sorts last
+  }
+
+  // Bitonic sort into "before" order (higher score, then smaller column).
+  constexpr int Mp = 32 * E;
+#pragma unroll
+  for (int size = 2; size <= Mp; size <<= 1) {
+#pragma unroll
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      if (stride >= 32) {  // partners in the same lane: registers e and e ^ (stride / 32)
+        const int es = stride / 32;
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+          if (e & es) continue;
+          const int pos = lane + 32 * e;                 // the lower element of the pair
+          const bool up = (pos & size) == 0;
+          const int f = e | es;
+          const bool swap = up ? before(sc[f], col[f], sc[e], col[e])
+                               : before(sc[e], col[e], sc[f], col[f]);
+          if (swap) {
+            const double ts = sc[e]; sc[e] = sc[f]; sc[f] = ts;
+            const int tc = col[e]; col[e] = col[f]; col[f] = tc;
+          }
+        }
+      } else {  // partners in lanes lane ^ stride, same register
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+          const double os = __shfl_xor_sync(0xffffffffu, sc[e], stride);
+          const int oc = __shfl_xor_sync(0xffffffffu, col[e], stride);
+          const int pos = lane + 32 * e;
+          const bool lower = (lane & stride) == 0;
+          const bool up = (pos & size) == 0;
+          // the lower element keeps the one that comes first in its run's order
+          const bool other_first = before(os, oc, sc[e], col[e]);
+          const bool take = (lower == up) ? other_first : !other_first;
+          if (take) {
+            sc[e] = os;
+            col[e] = oc;
+          }
+        }
+      }
+    }
+  }
+
+  const int keep = static_cast<int>(row_length(i, M, top_k, causal)) - 1;  // chosen besides i
+  marks[wl][lane] = 0u;
+  __syncwarp();
+#pragma unroll
+  for (int e = 0; e < E; ++e)
+    if (lane + 32 * e < keep) atomicOr(&marks[wl][col[e] >> 5], 1u << (col[e] & 31));
+  if (lane == 0) atomicOr(&marks[wl][i >> 5], 1u << (i & 31));
+  __syncwarp();
+  // Word `lane` holds columns 32 lane .. 32 lane + 31: ascending order by a warp scan.
+  uint32_t word = marks[wl][lane];
+  const int cnt = __popc(word);
+  int incl = cnt;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += v;
+  }
+  const long long row_start = bh * row_offset(M, M, top_k, causal) + row_offset(i, M, top_k, causal);
+  int pos = incl - cnt;
+  while (word) {
+    const int b = __ffs(word) - 1;
+    word &= word - 1;
+    col_idx[row_start + pos++] = lane * 32 + b;
+  }
+  if (lane == 0) {
+    row_ptr[r] = static_cast<int32_t>(row_start);
+    if (r == num_rows - 1)
+      row_ptr[num_rows] = static_cast<int32_t>(row_start + row_length(i, M, top_k, causal));
+  }
+}
+
+template <int E>
+int launch_select_warp(const double* qm, const double* kmT, int M, int d, int top_k, int causal,
+                       int32_t* row_ptr, int32_t* col_idx, long long rows, cudaStream_t s) {
+  const long long grid = (rows + kWarpRowsPerCta - 1) / kWarpRowsPerCta;
+  select_warp_kernel<E><<<static_cast<unsigned>(grid), 32 * kWarpRowsPerCta, 0, s>>>(
+      qm, kmT, M, d, top_k, causal, row_ptr, col_idx, rows);
+  return cudaGetLastError() == cudaSuccess ? BSA_OK : BSA_ERR_CUDA;
+}
+
 }  // namespace topk
 }  // namespace bsa
 
@@ -199,6 +342,17 @@ extern "C" int bsa_topk_pattern(const void* Q, const void* K, int BH, int N, int
   int Mp = 1;
   while (Mp < M) Mp <<= 1;
   if (Mp < 2) Mp = 2;
+  if (Mp <= 1024) {  // one warp per row, everything in registers
+    const int E = Mp <= 32 ? 1 : Mp / 32;
+    switch (E) {
+      case 1: return launch_select_warp<1>(qm, kmT, M, d, top_k, causal, row_ptr, col_idx, blocks, s);
+      case 2: return launch_select_warp<2>(qm, kmT, M, d, top_k, causal, row_ptr, col_idx, blocks, s);
+      case 4: return launch_select_warp<4>(qm, kmT, M, d, top_k, causal, row_ptr, col_idx, blocks, s);
+      case 8: return launch_select_warp<8>(qm, kmT, M, d, top_k, causal, row_ptr, col_idx, blocks, s);
+      case 16: return launch_select_warp<16>(qm, kmT, M, d, top_k, causal, row_ptr, col_idx, blocks, s);
+      default: return launch_select_warp<32>(qm, kmT, M, d, top_k, causal, row_ptr, col_idx, blocks, s);
+    }
+  }
   const size_t smem = static_cast<size_t>(Mp) * sizeof(double) + kMaxD * sizeof(double) +
                       static_cast<size_t>(Mp) * sizeof(int) + static_cast<size_t>(Mp);
   if (smem > 48 * 1024 &&

@@ -11,6 +11,7 @@
 """
 import math
 import os
+import pathlib
 
 import numpy as np
 import pytest
@@ -29,6 +30,9 @@ def _read_golden_rows(path):
         k, v = line.split(":")
         rows[int(k)] = [int(x) for x in v.split()]
     return rows
+
+
+GOLDEN_DIR = pathlib.Path(__file__).parent / "golden"
 
 
 def test_loglinear_matches_hand_enumeration(golden_dir):
@@ -187,6 +191,29 @@ def test_bigbird_rows_are_window_globals_and_the_drawn_columns():
     rows = [tuple(patterns.bigbird_cols(h, 20, M, w, (0,), R, seed)) for h in range(H)]
     assert len(set(rows)) > 1
     assert patterns.bigbird_cols(1, 20, M, w, (0,), 0, seed) == patterns.bigbird_cols(0, 20, M, w, (0,), 0, seed)
+
+
+def test_bigbird_row_worked_by_hand_from_published_outputs():
+    """Row i = 0 of head 0 with seed 0, M = 16, window 1, global block 5 and
+    three random draws.  Its keys are (0*16 + 0)*3 + r = 0, 1, 2, so the
+    draws are outputs 1, 2, 3 of the SplitMix64 stream at state 0, which
+    tests/golden/splitmix64_reference.txt gives from the published reference:
+        16294208416658607535, 7960286522194355700, 487617019471545679.
+    A column is floor(u * 16) with u = (output >> 11) / 2^53, i.e.
+    floor(output / 2^60): 14.13 -> 14, 6.90 -> 6, 0.42 -> 0.
+    The row is the window {0, 1}, the global column 5 and {14, 6, 0}."""
+    golden = {}
+    for line in open(GOLDEN_DIR / "splitmix64_reference.txt"):
+        if line.strip() and not line.startswith("#"):
+            state, outs = line.split(":")
+            golden[int(state)] = [int(x) for x in outs.split()]
+    outs = golden[0]
+    assert [o >> 60 for o in outs] == [14, 6, 0]   # the hand division above
+    assert [patterns.bigbird_random_col(0, 0, 0, r, 16, 3) for r in range(3)] == [14, 6, 0]
+    assert patterns.bigbird_cols(0, 0, 16, 1, (5,), 3, 0) == [0, 1, 5, 6, 14]
+    # the global row itself sees every block; another row gets column 5 too
+    assert patterns.bigbird_cols(0, 5, 16, 1, (5,), 3, 0) == list(range(16))
+    assert 5 in patterns.bigbird_cols(0, 9, 16, 1, (5,), 3, 0)
 
 
 def test_bigbird_random_columns_spread_over_the_row():

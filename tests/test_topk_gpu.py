@@ -41,6 +41,10 @@ CASES = [
     (1, 12, 3840, 64, 32, 10, True),
     (2, 5, 2048, 64, 32, 7, False),
     (1, 5, 3840, 128, 64, 3, True),
+    # the largest row one warp selects (1024 candidates), and a longer one
+    # that takes the one-CTA-per-row kernel (2048)
+    (1, 1, 32768, 64, 32, 50, False),
+    (1, 1, 65536, 64, 32, 20, True),
 ]
 
 
@@ -63,3 +67,17 @@ def test_topk_csr_bit_exact_and_forward_parity(case):
     err = np.abs(O.float().cpu().numpy() - Or)
     assert err.max() <= 2e-2 and err.mean() <= 2e-3
     assert np.abs(L.cpu().numpy() - Lr).max() <= 1e-3
+
+
+@pytest.mark.parametrize("N,bs", [(4096, 32), (65536, 32)])
+def test_topk_ties_go_to_the_smaller_column(N, bs):
+    """Constant K: every candidate of a row scores the same, so the row keeps
+    its smallest allowed columns -- in both selection kernels."""
+    B, H, d, k, causal = 1, 2, 64, 7, False
+    q, _, _ = workloads.make_qkv_shape(B, H, N, d, seed=5)
+    kk = torch.ones_like(q)
+    rp_d, ci_d = bsa.topk_pattern(q.cuda(), kk.cuda(), bs, k, causal)
+    torch.cuda.synchronize()
+    orp, oci = topk.topk_pattern(q.float().numpy(), kk.float().numpy(), bs, k, causal)
+    assert np.array_equal(rp_d.cpu().numpy(), orp)
+    assert np.array_equal(ci_d.cpu().numpy(), oci)
