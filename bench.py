@@ -57,9 +57,12 @@ KERNEL_DIR = os.path.join(ROOT, "block_sparse_attention_38_b200", "csrc")
 # (profiles/ holds the capture summaries).
 NCU_TRAFFIC = {
     "loglinear_4k": (25426944 + 0, "8fcc87898ba406ae"),
+    "local_global_8k": (284513280 + 48257536, "8fcc87898ba406ae"),
+    "bernoulli_4k": (201767680 + 49791744, "8fcc87898ba406ae"),
     "causal_loglinear_32k": (901510656 + 260866560, "8fcc87898ba406ae"),
+    "topk_4k": (25515776 + 0, "8fcc87898ba406ae"),
     # the decode kernel, keyed by the hash of DECODE_SOURCES
-    "decode_loglinear_32k": (175425792 + 3372544, "7be0c4ee875188a6"),
+    "decode_loglinear_32k": (175443200 + 3267584, "386e68dbdbbe3b74"),
     # the backward's three kernels together (dot + dK/dV + dQ), one backward
     "local_global_8k:backward": (134229248 + 4284160 + 336716800 + 111309568 + 330468096
                                  + 55514880, "418be616a808a425"),

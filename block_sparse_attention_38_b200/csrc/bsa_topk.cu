@@ -196,7 +196,7 @@ __global__ void __launch_bounds__(32 * kWarpRowsPerCta)
   // U columns c per round: all their loads are issued before the first of
   // their products, so one round costs one memory latency; the sums still
   // run over c in ascending order.
-  constexpr int U = 64 / E;  // 64 loads in flight per lane and round
+  constexpr int U = E >= 32 ? 1 : 32 / E;  // 32 loads in flight per lane and round
   for (int c0 = 0; c0 < d; c0 += U) {
     double qv[U], kv[U][E];
 #pragma unroll
