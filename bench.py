@@ -56,11 +56,11 @@ KERNEL_DIR = os.path.join(ROOT, "block_sparse_attention_38_b200", "csrc")
 # workload, valid only for the kernel sources whose sha256 prefix is given
 # (profiles/ holds the capture summaries).
 NCU_TRAFFIC = {
-    "loglinear_4k": (25426944 + 0, "8fcc87898ba406ae"),
-    "local_global_8k": (284513280 + 48257536, "8fcc87898ba406ae"),
-    "bernoulli_4k": (201767680 + 49791744, "8fcc87898ba406ae"),
-    "causal_loglinear_32k": (901510656 + 260866560, "8fcc87898ba406ae"),
-    "topk_4k": (25515776 + 0, "8fcc87898ba406ae"),
+    "loglinear_4k": (25431808 + 0, "91f71de28846c944"),
+    "local_global_8k": (286231296 + 49256960, "91f71de28846c944"),
+    "bernoulli_4k": (201685760 + 49137664, "91f71de28846c944"),
+    "causal_loglinear_32k": (928985856 + 261577984, "91f71de28846c944"),
+    "topk_4k": (25515264 + 0, "91f71de28846c944"),
     # the decode kernel, keyed by the hash of DECODE_SOURCES
     "decode_loglinear_32k": (175443200 + 3267584, "386e68dbdbbe3b74"),
     # the backward's three kernels together (dot + dK/dV + dQ), one backward

@@ -51,12 +51,17 @@ constexpr int kThreads = 32 * kWarps;
 constexpr int kProdWarp = 8;                // producer of slot s is warp kProdWarp + 2 s
 constexpr int kMmaWarp = 9;
 constexpr int kTiRing = 3;                  // tile-info entries per slot
-// One group of 4 probabilities in kPolyEvery is computed by a polynomial on
-// the FMA pipe instead of the MUFU ex2 (0: all by ex2), to relieve the MUFU.
+// For d = 128, one group of 4 probabilities in kPolyEvery is computed by a
+// polynomial on the FMA pipe instead of the MUFU ex2, to relieve the MUFU
+// (measured: 947 -> 900 us on causal_loglinear_32k).  For d = 64 the steps
+// have half the tensor work and the polynomial's extra instructions cost
+// more than the MUFU time they save (727 -> 752 us on bernoulli_4k, 78 -> 82
+// us on loglinear_4k), so every exponential there is an ex2.
 #ifndef BSA_POLY_EVERY
 #define BSA_POLY_EVERY 4
 #endif
-constexpr int kPolyEvery = BSA_POLY_EVERY;
+template <int D>
+__host__ __device__ constexpr int poly_every() { return D == 64 ? 0 : BSA_POLY_EVERY; }
 
 constexpr int kMaxGrid = 160;               // CTAs per launch (the host caps the grid)
 constexpr int kMaxVirt = kSlots * kMaxGrid; // slots scheduled as workers
@@ -960,7 +965,8 @@ __device__ void softmax_role(int s, const FwdArgs& a, Ctrl* ctl, const uint32_t*
               fma2(d0, d1, sl2, nmu);              // scaled score minus the maximum
               fma2(d2, d3, sl2, nmu);
               float p0, p1, p2, p3;
-              if (kPolyEvery > 0 && (c / 4) % (kPolyEvery > 0 ? kPolyEvery : 1) == kPolyEvery - 1) {
+              constexpr int kPoly = poly_every<D>();
+              if (kPoly > 0 && (c / 4) % (kPoly > 0 ? kPoly : 1) == kPoly - 1) {
                 exp2_poly2(d0, d1);                // this share of 2^x on the FMA pipe
                 exp2_poly2(d2, d3);
                 p0 = d0; p1 = d1; p2 = d2; p3 = d3;

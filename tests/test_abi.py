@@ -188,3 +188,28 @@ def test_forward_rejects_bad_arguments_without_launching():
     assert call(d=96) == bsa.ERR_UNSUPPORTED
     assert call(bs=16, N=256) == bsa.ERR_UNSUPPORTED
     assert call(N=32 * 4097) == bsa.ERR_UNSUPPORTED              # M above the supported maximum
+
+
+def test_forward_ws_rejects_bad_arguments_and_sizes_its_workspace():
+    """bsa_forward_ws checks its workspace pointer before any CUDA call, and
+    bsa_forward_workspace_bytes is the closed form of its layout: 320 chunk
+    slots, four 8-byte count words each, then per slot 128 (m, l) pairs of
+    fp32 and a d x 128 fp32 block of O."""
+    lib = bsa.library()
+    P = 1 << 20
+    base = dict(Q=P, K=P, V=P, rp=P, ci=P, B=1, H=2, N=256, d=64, bs=32, scale=0.125, causal=0,
+                O=P, L=P, ws=P, nbytes=1 << 24)
+
+    def call(**kw):
+        a = dict(base, **kw)
+        return lib.bsa_forward_ws(a["Q"], a["K"], a["V"], a["rp"], a["ci"], a["B"], a["H"],
+                                  a["N"], a["d"], a["bs"], a["scale"], a["causal"], a["O"], a["L"],
+                                  a["ws"], a["nbytes"], None)
+
+    assert call(ws=P + 8) == bsa.ERR_INVALID_ARG                  # misaligned workspace
+    assert call(Q=None) == bsa.ERR_INVALID_ARG
+    assert call(N=250) == bsa.ERR_INVALID_ARG
+    assert call(d=96) == bsa.ERR_UNSUPPORTED
+    for d in (64, 128):
+        assert bsa.forward_workspace_bytes(d) == 320 * 4 * 8 + 320 * (128 * 8 + 128 * d * 4)
+    assert bsa.forward_workspace_bytes(32) == 0
