@@ -73,15 +73,15 @@ bool device_info(int dev, DeviceInfo* out) {
   return true;
 }
 
-// Raises the dynamic shared-memory limit of the <BS, D> kernel on `dev` to
-// `bytes` once per instantiation and device, under the device mutex.
-template <int BS, int D>
+// Raises the dynamic shared-memory limit of the <BS, D, POS> kernel on `dev`
+// to `bytes` once per instantiation and device, under the device mutex.
+template <int BS, int D, bool POS>
 bool ensure_smem_attr(int dev, int bytes) {
   static int set_bytes[64] = {};
   if (dev < 0 || dev >= 64) return false;
   std::lock_guard<std::mutex> lock(device_mutex());
   if (set_bytes[dev] >= bytes) return true;
-  if (cudaFuncSetAttribute(pp::fwd_kernel<BS, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  if (cudaFuncSetAttribute(pp::fwd_kernel<BS, D, POS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            bytes) != cudaSuccess)
     return false;
   set_bytes[dev] = bytes;
@@ -145,10 +145,17 @@ int launch_fwd(const void* Q, const void* K, const void* V, const int32_t* row_p
   // stages, control block, the tile-bitmap buffers, and 1024 bytes of alignment slack
   const int smem = C::OFF_CTRL + static_cast<int>(sizeof(pp::Ctrl)) +
                    pp::kSlots * pp::kTiRing * pp::bitmap_words<BS>(a.W) * 4 + 1024;
-  if (!ensure_smem_attr<BS, D>(dev, smem)) return BSA_ERR_CUDA;
   long long grid = a.num_tiles < di.sms ? a.num_tiles : di.sms;
   if (grid > pp::kMaxGrid) grid = pp::kMaxGrid;
-  pp::fwd_kernel<BS, D><<<static_cast<unsigned>(grid), pp::kThreads, smem, stream>>>(tq, tk, tv, a);
+  // One instantiation per sign of the scale: each kernel carries only the
+  // row-maximum code (maximum or minimum of the raw scores) it runs.
+  if (a.scale_log2 > 0.f) {
+    if (!ensure_smem_attr<BS, D, true>(dev, smem)) return BSA_ERR_CUDA;
+    pp::fwd_kernel<BS, D, true><<<static_cast<unsigned>(grid), pp::kThreads, smem, stream>>>(tq, tk, tv, a);
+  } else {
+    if (!ensure_smem_attr<BS, D, false>(dev, smem)) return BSA_ERR_CUDA;
+    pp::fwd_kernel<BS, D, false><<<static_cast<unsigned>(grid), pp::kThreads, smem, stream>>>(tq, tk, tv, a);
+  }
   if (cudaGetLastError() != cudaSuccess) return BSA_ERR_CUDA;
   return BSA_OK;
 }

@@ -817,7 +817,7 @@ __device__ __forceinline__ void chunk_epilogue(const FwdArgs& a, const TileInfo&
 // pairs) goes to the slot's P columns; at the end of the tile O / l and the
 // LSE are stored.  Every TMEM access here waits for itself inside one asm
 // statement (see sm100_ptx.cuh).
-template <int BS, int D>
+template <int BS, int D, bool POS>
 __device__ void softmax_role(int s, const FwdArgs& a, Ctrl* ctl, const uint32_t* bitmaps,
                              uint32_t tmem) {
   using C = Cfg<BS, D>;
@@ -897,7 +897,7 @@ __device__ void softmax_role(int s, const FwdArgs& a, Ctrl* ctl, const uint32_t*
         // minimum for a negative scale); on the diagonal block of a causal
         // tile, keys after the query are first set to the value that scales
         // to -inf.
-        const bool pos = sl2 > 0.f;
+        constexpr bool pos = POS;                // the scale's sign, a template parameter
         const float sentinel = pos ? kNegInf : INFINITY;
         float hraw = sentinel;
 #pragma unroll
@@ -909,7 +909,7 @@ __device__ void softmax_role(int s, const FwdArgs& a, Ctrl* ctl, const uint32_t*
               if ((64 * h + gi * 32 + c) % BS > qq) x[gi * 32 + c] = sentinel;
           }
           float ma = sentinel, mb = sentinel;
-          if (pos) {
+          if constexpr (pos) {
 #pragma unroll
             for (int c = 0; c < 32; c += 4) {
               ma = max3f(ma, x[gi * 32 + c], x[gi * 32 + c + 1]);
@@ -1061,7 +1061,7 @@ __device__ void softmax_role(int s, const FwdArgs& a, Ctrl* ctl, const uint32_t*
   }
 }
 
-template <int BS, int D>
+template <int BS, int D, bool POS>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const FwdArgs args) {
@@ -1109,7 +1109,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = ctl->tmem_base;
 
   if (warp < 4 * kSlots) {
-    softmax_role<BS, D>(warp >> 2, args, ctl, bitmaps, tmem);
+    softmax_role<BS, D, POS>(warp >> 2, args, ctl, bitmaps, tmem);
     __syncwarp();
   } else if (warp == kProdWarp || warp == kProdWarp + 2) {
     produce_role<BS, D>((warp - kProdWarp) >> 1, &tmQ, &tmK, &tmV, args, smem, ctl, bitmaps);
