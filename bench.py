@@ -56,11 +56,11 @@ KERNEL_DIR = os.path.join(ROOT, "block_sparse_attention_38_b200", "csrc")
 # workload, valid only for the kernel sources whose sha256 prefix is given
 # (profiles/ holds the capture summaries).
 NCU_TRAFFIC = {
-    "loglinear_4k": (25431808 + 0, "91f71de28846c944"),
-    "local_global_8k": (286231296 + 49256960, "91f71de28846c944"),
-    "bernoulli_4k": (201685760 + 49137664, "91f71de28846c944"),
-    "causal_loglinear_32k": (928985856 + 261577984, "91f71de28846c944"),
-    "topk_4k": (25515264 + 0, "91f71de28846c944"),
+    "loglinear_4k": (25427712 + 0, "b3f14ca92b384dc0"),
+    "local_global_8k": (286169856 + 48533248, "b3f14ca92b384dc0"),
+    "bernoulli_4k": (201544448 + 49105152, "b3f14ca92b384dc0"),
+    "causal_loglinear_32k": (876655360 + 254986752, "b3f14ca92b384dc0"),
+    "topk_4k": (25511680 + 0, "b3f14ca92b384dc0"),
     # the decode kernel, keyed by the hash of DECODE_SOURCES
     "decode_loglinear_32k": (175443200 + 3267584, "386e68dbdbbe3b74"),
     # the backward's three kernels together (dot + dK/dV + dQ), one backward
