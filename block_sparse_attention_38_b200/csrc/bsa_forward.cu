@@ -73,15 +73,15 @@ bool device_info(int dev, DeviceInfo* out) {
   return true;
 }
 
-// Raises the dynamic shared-memory limit of the <BS, D, POS> kernel on `dev`
-// to `bytes` once per instantiation and device, under the device mutex.
-template <int BS, int D, bool POS>
+// Raises the dynamic shared-memory limit of the <BS, D, POS, CAUSAL> kernel
+// on `dev` to `bytes` once per instantiation and device, under the device mutex.
+template <int BS, int D, bool POS, bool CAUSAL>
 bool ensure_smem_attr(int dev, int bytes) {
   static int set_bytes[64] = {};
   if (dev < 0 || dev >= 64) return false;
   std::lock_guard<std::mutex> lock(device_mutex());
   if (set_bytes[dev] >= bytes) return true;
-  if (cudaFuncSetAttribute(pp::fwd_kernel<BS, D, POS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  if (cudaFuncSetAttribute(pp::fwd_kernel<BS, D, POS, CAUSAL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            bytes) != cudaSuccess)
     return false;
   set_bytes[dev] = bytes;
@@ -147,14 +147,23 @@ int launch_fwd(const void* Q, const void* K, const void* V, const int32_t* row_p
                    pp::kSlots * pp::kTiRing * pp::bitmap_words<BS>(a.W) * 4 + 1024;
   long long grid = a.num_tiles < di.sms ? a.num_tiles : di.sms;
   if (grid > pp::kMaxGrid) grid = pp::kMaxGrid;
-  // One instantiation per sign of the scale: each kernel carries only the
-  // row-maximum code (maximum or minimum of the raw scores) it runs.
-  if (a.scale_log2 > 0.f) {
-    if (!ensure_smem_attr<BS, D, true>(dev, smem)) return BSA_ERR_CUDA;
-    pp::fwd_kernel<BS, D, true><<<static_cast<unsigned>(grid), pp::kThreads, smem, stream>>>(tq, tk, tv, a);
+  // One instantiation per sign of the scale and per causal flag: each kernel
+  // carries only the row-maximum code (maximum or minimum of the raw scores)
+  // and the diagonal masking it runs.
+  const unsigned g = static_cast<unsigned>(grid);
+  const bool pos = a.scale_log2 > 0.f;
+  if (pos && causal) {
+    if (!ensure_smem_attr<BS, D, true, true>(dev, smem)) return BSA_ERR_CUDA;
+    pp::fwd_kernel<BS, D, true, true><<<g, pp::kThreads, smem, stream>>>(tq, tk, tv, a);
+  } else if (pos) {
+    if (!ensure_smem_attr<BS, D, true, false>(dev, smem)) return BSA_ERR_CUDA;
+    pp::fwd_kernel<BS, D, true, false><<<g, pp::kThreads, smem, stream>>>(tq, tk, tv, a);
+  } else if (causal) {
+    if (!ensure_smem_attr<BS, D, false, true>(dev, smem)) return BSA_ERR_CUDA;
+    pp::fwd_kernel<BS, D, false, true><<<g, pp::kThreads, smem, stream>>>(tq, tk, tv, a);
   } else {
-    if (!ensure_smem_attr<BS, D, false>(dev, smem)) return BSA_ERR_CUDA;
-    pp::fwd_kernel<BS, D, false><<<static_cast<unsigned>(grid), pp::kThreads, smem, stream>>>(tq, tk, tv, a);
+    if (!ensure_smem_attr<BS, D, false, false>(dev, smem)) return BSA_ERR_CUDA;
+    pp::fwd_kernel<BS, D, false, false><<<g, pp::kThreads, smem, stream>>>(tq, tk, tv, a);
   }
   if (cudaGetLastError() != cudaSuccess) return BSA_ERR_CUDA;
   return BSA_OK;

@@ -817,7 +817,7 @@ __device__ __forceinline__ void chunk_epilogue(const FwdArgs& a, const TileInfo&
 // pairs) goes to the slot's P columns; at the end of the tile O / l and the
 // LSE are stored.  Every TMEM access here waits for itself inside one asm
 // statement (see sm100_ptx.cuh).
-template <int BS, int D, bool POS>
+template <int BS, int D, bool POS, bool CAUSAL>
 __device__ void softmax_role(int s, const FwdArgs& a, Ctrl* ctl, const uint32_t* bitmaps,
                              uint32_t tmem) {
   using C = Cfg<BS, D>;
@@ -869,7 +869,7 @@ __device__ void softmax_role(int s, const FwdArgs& a, Ctrl* ctl, const uint32_t*
         const int jb = it.next();
         const uint32_t gm = ((1u << GPB) - 1u) << (b * GPB);
         if (row_ok && jb >= 0 && ((bm[sub * W + (jb >> 5)] >> (jb & 31)) & 1u)) own |= gm;
-        if (a.causal && jb == r_sub) diag |= gm;
+        if (CAUSAL && jb == r_sub) diag |= gm;  // CAUSAL: a template parameter equal to a.causal
       }
       diag &= own;
       if (!warp_wait(&B.s_full, s_seen & 1, &ctl->abort)) return;
@@ -1061,7 +1061,7 @@ __device__ void softmax_role(int s, const FwdArgs& a, Ctrl* ctl, const uint32_t*
   }
 }
 
-template <int BS, int D, bool POS>
+template <int BS, int D, bool POS, bool CAUSAL>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const FwdArgs args) {
@@ -1109,7 +1109,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = ctl->tmem_base;
 
   if (warp < 4 * kSlots) {
-    softmax_role<BS, D, POS>(warp >> 2, args, ctl, bitmaps, tmem);
+    softmax_role<BS, D, POS, CAUSAL>(warp >> 2, args, ctl, bitmaps, tmem);
     __syncwarp();
   } else if (warp == kProdWarp || warp == kProdWarp + 2) {
     produce_role<BS, D>((warp - kProdWarp) >> 1, &tmQ, &tmK, &tmV, args, smem, ctl, bitmaps);
