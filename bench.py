@@ -59,7 +59,7 @@ NCU_TRAFFIC = {
     "loglinear_4k": (25427712 + 0, "b3f14ca92b384dc0"),
     "local_global_8k": (286169856 + 48533248, "b3f14ca92b384dc0"),
     "bernoulli_4k": (201544448 + 49105152, "b3f14ca92b384dc0"),
-    "causal_loglinear_32k": (876655360 + 254986752, "b3f14ca92b384dc0"),
+    "causal_loglinear_32k": (848413184 + 254313728, "e360f7440fb5438f"),
     "topk_4k": (25511680 + 0, "b3f14ca92b384dc0"),
     # the decode kernel, keyed by the hash of DECODE_SOURCES
     "decode_loglinear_32k": (175443200 + 3267584, "386e68dbdbbe3b74"),
