@@ -158,9 +158,10 @@ int bsa_forward(const void* Q, const void* K, const void* V,
  * bsa_forward_ws -- bsa_forward with a workspace for chunked tiles.
  *
  * The kernel's unit of work is a tile of 128 query rows walking the union of
- * its block rows' columns.  When one tile's walk is longer than an even share
- * of the whole launch per tile slot (a global row, a long causal row), its
- * walk is cut into chunks that run as separate units; each chunk leaves its
+ * its block rows' columns.  When one tile's walk is longer than two even
+ * shares of the whole launch per tile slot (a global row on a small problem,
+ * say), its walk is cut into chunks that run as separate units; each chunk
+ * leaves its
  * unnormalised O and its (max, sum) statistics in the workspace and the last
  * chunk of the tile to finish merges them, weighting chunk c by
  * exp(m_c - max_c m_c) ("split long rows into kv-chunks"; the merged softmax
