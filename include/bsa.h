@@ -161,9 +161,8 @@ int bsa_forward(const void* Q, const void* K, const void* V,
  * its block rows' columns.  When one tile's walk is longer than two even
  * shares of the whole launch per tile slot (a global row on a small problem,
  * say), its walk is cut into chunks that run as separate units; each chunk
- * leaves its
- * unnormalised O and its (max, sum) statistics in the workspace and the last
- * chunk of the tile to finish merges them, weighting chunk c by
+ * leaves its unnormalised O and its (max, sum) statistics in the workspace
+ * and the last chunk of the tile to finish merges them, weighting chunk c by
  * exp(m_c - max_c m_c) ("split long rows into kv-chunks"; the merged softmax
  * is the one of section 3.3 of "Block Sparse Attention with Log-Linear
  * Complexity" over the union of the chunks' keys).  The result is the same
